@@ -1,0 +1,264 @@
+"""Pins for the fp64 oracle, each against something other than the oracle itself.
+
+The pages print no worked example, so the pins are: library routines the method reduces to in a
+special case (scaled-dot-product attention, a lexicographic sort, torch's FP8 decoding), closed
+forms of hand-built cases, and invariants of the definition. Every test runs on the CPU.
+Definitions followed: "HySparse2: How Xiaomi Split the Transformer to Fix Agent Prefill Costs",
+section "KV Reuse and Token-Level Sparse Selection" (full layer -> KV cache + token indices;
+1,024 tokens + forced window of the 128 most recent; sparse layers reuse both).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from workloads import Workload, bf16_bits_to_f32, f32_to_bf16_bits
+
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def small(seed=3, **kw):
+    cfg = dict(name="small", batch=2, n_q=1, n_heads=4, n_sparse=2, kv_dtype="bf16",
+               lengths=(300, 517), needles=4, topk=64, window=16)
+    cfg.update(kw)
+    return W.make_workload(cfg, seed=seed)
+
+
+def dense_f64(w, which):
+    """Cache K or V widened to float64 through torch's own decoders (bf16 / float8_e4m3fn)."""
+    a = w.k if which == "k" else w.v
+    if w.kv_dtype == "bf16":
+        return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).double()
+    sc = w.k_scale if which == "k" else w.v_scale
+    x = torch.from_numpy(a.copy()).view(torch.float8_e4m3fn).double()
+    return x * torch.from_numpy(sc).double()[:, None]
+
+
+def q_f64(q):
+    return torch.from_numpy(q.view(np.int16).copy()).view(torch.bfloat16).double()
+
+
+def sdpa_row(w, q_row, b, idx, scale):
+    """torch SDPA (float64, CPU) of one query row's H heads over cache positions idx of seq b."""
+    K = dense_f64(w, "k")[w.kv_start[b] + torch.as_tensor(idx)]
+    V = dense_f64(w, "v")[w.kv_start[b] + torch.as_tensor(idx)]
+    H = q_row.shape[0]
+    qq = q_row[None, :, None, :]                       # [1, H, 1, d]
+    kk = K[None, None].expand(1, H, -1, -1)
+    vv = V[None, None].expand(1, H, -1, -1)
+    return torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)[0, :, 0]
+
+
+# ------------------------------------------------------------------ formats
+
+def test_e4m3_table_matches_torch(oracle_lib):
+    tab = oracle_lib.e4m3_table()
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(tab), nan)
+    assert np.array_equal(tab[~nan], ref[~nan])
+    assert tab[0x7E] == 448.0 and tab[0x01] == 2.0 ** -9
+
+
+# ------------------------------------------------------------------ full attention
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("n_q", [1, 5])
+def test_full_attention_matches_sdpa(oracle_lib, kv_dtype, n_q):
+    w = small(kv_dtype=kv_dtype, n_q=n_q)
+    c = 1.0 / math.sqrt(w.head_dim)
+    o, lse, s = oracle_lib.full_attn(w)
+    q = q_f64(w.q_full)
+    for r in range(w.n_rows):
+        b, i = divmod(r, w.n_q)
+        p = w.position(b, i)
+        ref = sdpa_row(w, q[b, i], b, np.arange(p + 1), c).numpy()
+        np.testing.assert_allclose(o[r], ref, rtol=0, atol=1e-12)
+
+
+def test_single_head_scores_are_softmax_weights(oracle_lib):
+    """Hq = 1: s[t] is the softmax weight of t; SDPA with V = identity rows exposes it."""
+    w = small(n_heads=1, lengths=(40, 77), needles=0)
+    c = 1.0 / math.sqrt(w.head_dim)
+    _, lse, s = oracle_lib.full_attn(w)
+    q = q_f64(w.q_full)
+    for b in range(w.batch):
+        p = w.position(b, 0)
+        K = dense_f64(w, "k")[w.kv_start[b]:w.kv_start[b] + p + 1]
+        eye = torch.eye(p + 1, dtype=torch.float64)
+        wts = torch.nn.functional.scaled_dot_product_attention(
+            q[b, 0, 0][None, None, None], K[None, None], eye[None, None], scale=c)[0, 0, 0]
+        np.testing.assert_allclose(s[b, :p + 1], wts.numpy(), rtol=1e-12, atol=0)
+
+
+def test_constant_value_rows_give_that_row(oracle_lib):
+    w = small(needles=0)
+    row = f32_to_bf16_bits(np.linspace(-2, 2, w.head_dim, dtype=np.float32))
+    w.v = np.tile(row, (w.kv_rows, 1))
+    o, _, _ = oracle_lib.full_attn(w, want_scores=False)
+    np.testing.assert_allclose(o, np.broadcast_to(bf16_bits_to_f32(row), o.shape),
+                               rtol=1e-13, atol=1e-13)
+
+
+def hand_case(T=4, H=2):
+    """d = 4, so c = 1/2 exactly; q_h = (2, 0, 0, 0) for every head; k_t = (t, 0, 0, 0).
+    Logits are l[t] = t, weights e^t / sum_j e^j, lse = log sum_j e^j."""
+    d = 4
+    k = np.zeros((T, d), np.float32)
+    k[:, 0] = np.arange(T)
+    v = np.zeros((T, d), np.float32)
+    v[:, 1] = np.arange(T) * 0.5
+    v[:, 2] = 1.0
+    q = np.zeros((1, 1, H, d), np.float32)
+    q[..., 0] = 2.0
+    return Workload(name="hand", seed=0, batch=1, n_q=1, n_heads=H, head_dim=d, n_sparse=1,
+                    kv_dtype="bf16", topk=1, window=1,
+                    kv_len=np.array([T], np.int32), kv_start=np.array([0], np.int64),
+                    k=f32_to_bf16_bits(k), v=f32_to_bf16_bits(v), k_scale=None, v_scale=None,
+                    q_full=f32_to_bf16_bits(q), q_sparse=f32_to_bf16_bits(q[None]),
+                    needle_pos=[np.zeros(0, np.int64)], needle_row=[np.zeros(0, np.int64)])
+
+
+def test_hand_case_closed_form(oracle_lib):
+    T, H = 4, 2
+    w = hand_case(T, H)
+    o, lse, s = oracle_lib.full_attn(w, scale=0.5)
+    Z = sum(math.exp(t) for t in range(T))
+    wt = np.array([math.exp(t) / Z for t in range(T)])
+    assert np.allclose(lse, math.log(Z), rtol=1e-15)
+    assert np.allclose(o[0, :, 1], (wt * 0.5 * np.arange(T)).sum(), rtol=1e-15)
+    assert np.allclose(o[0, :, 2], 1.0, rtol=1e-15)
+    assert np.allclose(o[0, :, [0, 3]], 0.0)
+    np.testing.assert_allclose(s[0, :T], H * wt, rtol=1e-14)
+    # top-1 of candidates [0, 3) is t = 2; the window of 1 is {3}
+    assert oracle_lib.select_f64(s[0, :T], T - 1, 1, 1).tolist() == [2, 3]
+
+
+def test_identical_keys_give_uniform_scores(oracle_lib):
+    w = small(needles=0, n_q=3)
+    w.k = np.tile(w.k[:1], (w.kv_rows, 1))
+    _, lse, s = oracle_lib.full_attn(w)
+    for r in range(w.n_rows):
+        p = w.position(*divmod(r, w.n_q))
+        np.testing.assert_allclose(s[r, :p + 1], w.n_heads / (p + 1), rtol=1e-13)
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+def test_scores_sum_to_heads_and_are_bounded(oracle_lib, kv_dtype):
+    w = small(kv_dtype=kv_dtype, n_q=4)
+    _, _, s = oracle_lib.full_attn(w)
+    for r in range(w.n_rows):
+        p = w.position(*divmod(r, w.n_q))
+        row = s[r, :p + 1]
+        assert abs(row.sum() - w.n_heads) <= 1e-12 * w.n_heads
+        assert row.min() >= 0 and row.max() <= w.n_heads
+
+
+# ------------------------------------------------------------------ selection
+
+def brute_select(s, p, k, w):
+    nc = max(0, p - w + 1)
+    if nc <= k:
+        return np.arange(p + 1)
+    t = np.arange(nc)
+    order = np.lexsort((t, -s[:nc]))          # score descending, then index ascending
+    return np.concatenate([np.sort(order[:k]), np.arange(nc, p + 1)])
+
+
+@pytest.mark.parametrize("k,win", [(8, 4), (3, 1), (1024, 128), (64, 16)])
+def test_selection_matches_lexsort(oracle_lib, k, win):
+    rng = np.random.default_rng(11)
+    for p in list(range(0, 40)) + [127, 128, 129, 1150, 1151, 1152, 1153, 2047]:
+        for kind in ("cont", "ties"):
+            s = rng.random(p + 1)
+            if kind == "ties":
+                s = np.round(s * 4) / 4              # heavy ties
+            ref = brute_select(s, p, k, win)
+            got = oracle_lib.select_f64(s, p, k, win)
+            assert np.array_equal(got, ref), (p, kind)
+            got32 = oracle_lib.select_f32(s.astype(np.float32), p, k, win)
+            ref32 = brute_select(s.astype(np.float32).astype(np.float64), p, k, win)
+            assert np.array_equal(got32, ref32), (p, kind)
+
+
+def test_selection_all_equal_takes_lowest_indices(oracle_lib):
+    p, k, win = 5000, 1024, 128
+    got = oracle_lib.select_f64(np.ones(p + 1), p, k, win)
+    assert np.array_equal(got, np.concatenate([np.arange(k), np.arange(p - win + 1, p + 1)]))
+
+
+def test_selection_f32_uses_bit_order(oracle_lib):
+    # adjacent floats differ only in the last bit; denormals and +0 are ordered too
+    vals = np.array([0.0, 1e-45, 2e-45, 1.0, np.nextafter(np.float32(1), np.float32(2))],
+                    dtype=np.float32)
+    s = np.concatenate([vals, np.zeros(4, np.float32)])
+    got = oracle_lib.select_f32(s, s.size - 1, 2, 4)
+    assert got.tolist() == [3, 4, 5, 6, 7, 8]
+
+
+def check_selection_invariants(idx, count, p, k, win):
+    S = idx[:count]
+    assert count == min(p + 1, k + win)
+    assert np.all(np.diff(S) > 0) and S[0] >= 0 and S[-1] <= p
+    wlo = max(0, p - win + 1)
+    assert set(range(wlo, p + 1)) <= set(S.tolist())
+
+
+def test_block_invariants_and_needles(oracle_lib):
+    w = W.make_workload(0)            # 4,096-token decode, 16 heads, 8 needles
+    out = oracle_lib.block(w)
+    p = w.position(0, 0)
+    check_selection_invariants(out["idx"][0], out["count"][0], p, w.topk, w.window)
+    assert set(w.needle_pos[0].tolist()) <= set(out["idx"][0, :out["count"][0]].tolist())
+
+
+def test_needles_selected_in_chunk_rows(oracle_lib):
+    w = small(n_q=6, lengths=(2000, 2600), needles=6, topk=64, window=16)
+    out = oracle_lib.block(w)
+    for b in range(w.batch):
+        for t, i in zip(w.needle_pos[b], w.needle_row[b]):
+            r = b * w.n_q + int(i)
+            sel = out["idx"][r, :out["count"][r]]
+            assert int(t) in set(sel.tolist())
+
+
+# ------------------------------------------------------------------ sparse attention
+
+def test_full_budget_sparse_equals_full(oracle_lib):
+    """When topk + window covers [0, p], the sparse layer is full causal attention."""
+    w = small(n_q=3, topk=600, window=16)
+    rows = np.arange(w.n_rows)
+    o_full, _, s = oracle_lib.full_attn(w)
+    idx, count = oracle_lib.select_rows(w, rows, s)
+    for r in rows:
+        assert count[r] == w.position(*divmod(r, w.n_q)) + 1
+    o_sp = oracle_lib.sparse_attn(w, w.q_full, rows, idx, count)
+    assert np.array_equal(o_sp, o_full)
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+def test_sparse_matches_sdpa_over_selected_rows(oracle_lib, kv_dtype):
+    w = small(kv_dtype=kv_dtype, n_q=2, topk=32, window=8)
+    c = 1.0 / math.sqrt(w.head_dim)
+    out = oracle_lib.block(w)
+    q = q_f64(w.q_sparse[1])
+    for r in range(w.n_rows):
+        b, i = divmod(r, w.n_q)
+        sel = out["idx"][r, :out["count"][r]]
+        ref = sdpa_row(w, q[b, i], b, sel, c).numpy()
+        np.testing.assert_allclose(out["o_sparse"][1][r], ref, rtol=0, atol=1e-12)
+
+
+def test_planted_mistake_is_caught(oracle_lib):
+    """A plausible slip -- selecting inside the window or dropping the forced window -- must
+    fail the lexsort pin; checked by perturbing the oracle's output on the CPU."""
+    rng = np.random.default_rng(5)
+    p, k, win = 300, 32, 8
+    s = rng.random(p + 1)
+    ref = brute_select(s, p, k, win)
+    got = oracle_lib.select_f64(s, p, k, win)
+    assert np.array_equal(got, ref)
+    wrong = np.sort(np.lexsort((np.arange(p + 1), -s))[:k + win])   # window not forced
+    assert not np.array_equal(wrong, ref)
