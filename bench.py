@@ -1,0 +1,366 @@
+"""Benchmark of the HySparse2 hybrid-block decode step on B200.
+
+`python bench.py --gpus N --steps K --warmup W [--impl hs2|reference] [--config C]`
+
+One step = one hybrid block over one batch of synthetic decode queries: the full-attention
+layer (pass 1: output + log-sum-exp; pass 2: importance scores), the token top-k + forced
+window selection, and every sparse layer, all through `hs2_block_decode` (C ABI). The default
+workload is the 128k-context decode batch: 8 sequences with contexts drawn uniformly from
+65,536..131,072 tokens, 32 query heads on one bf16 K/V head, 3 sparse layers, top-1,024 +
+window 128. Its K/V cache (~400 MB) is larger than the 126 MB L2, so no flush is needed
+between steps.
+
+Multi-GPU (torchrun): every rank runs its own batch (independent sequences, no exchange);
+`value` is all ranks' tokens over the slowest rank's time (weak scaling).
+`--impl reference` times the fp64 CPU oracle on the same workload (rank 0 only).
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "hybrid-block decode tokens/s at 128k/1M ctx; achieved % of HBM roofline"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="hs2", choices=["hs2", "reference"])
+    ap.add_argument("--config", type=int, default=1, help="workload id (0..2 decode)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    a.steps = max(a.steps, 1)
+    return a
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def algorithmic_bytes(w) -> dict:
+    """Bytes each step must move at least once, per kernel (see the design notes):
+    pass 1 reads K and V of every cached token once; pass 2 reads K again and writes one fp32
+    score per token; the selection reads every score once; each sparse layer gathers
+    topk + window K/V rows per query. Queries, outputs, lse and indices are counted too."""
+    T = int(w.kv_len.astype(np.int64).sum())
+    H, d, B = w.n_heads, w.head_dim, w.batch
+    elem = 2 if w.kv_dtype == "bf16" else 1
+    row = d * elem + (4 if w.kv_dtype == "fp8" else 0)          # one K (or V) row + scale
+    q = B * H * d * 2
+    o = B * H * d * 4
+    p1 = T * 2 * row + q + o + B * H * 4
+    p2 = T * row + T * 4 + q + B * H * 4
+    tk = T * 4 + B * (w.topk + w.window) * 4
+    sel = [min(int(t), w.topk + w.window) for t in w.kv_len]
+    sp = sum(sel) * 2 * row + q + o + sum(sel) * 4
+    return dict(pass1=p1, pass2=p2, topk=tk, sparse=sp, total=p1 + p2 + tk + w.n_sparse * sp)
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _poll(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(0.005)
+
+    def sample(self):
+        if self.nv is None:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for b, name in self.REASONS.items():
+                if bits & b and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        self.t = threading.Thread(target=self._poll, daemon=True)
+        self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self.t.join()
+        self.sample()
+
+    def result(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(a):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_baseline(w, budget_s=20.0):
+    """The oracle as it stands, on the host cores, over whole batches of the same workload."""
+    import oracle
+    oracle.build()
+    rows = np.arange(w.n_rows)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.block(w, rows=rows)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el > budget_s * 0.5 or reps >= 3:
+            break
+    tok = reps * w.n_rows
+    return {"value": tok / el, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{reps} full batch(es) of {w.n_rows} decode queries (all "
+                      f"{int(w.kv_len.sum())} cached tokens, all layers), {el:.1f} s"}
+
+
+def run_reference(a, w):
+    world, rank, _ = dist_setup(a)
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    rows = np.arange(w.n_rows)
+    for _ in range(a.warmup if a.warmup <= 3 else 3):
+        oracle.block(w, rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        oracle.block(w, rows=rows)
+    el = time.perf_counter() - t0
+    value = a.steps * w.n_rows / el
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": el / a.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: the full batch of {w.n_rows} decode queries"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": w.name, "batch": w.batch, "queries_per_seq": w.n_q,
+            "context_tokens_total": int(w.kv_len.astype(np.int64).sum()),
+            "context_min": int(w.kv_len.min()), "context_max": int(w.kv_len.max()),
+            "n_heads": w.n_heads, "kv_heads": 1, "head_dim": w.head_dim,
+            "n_sparse_layers": w.n_sparse, "topk": w.topk, "window": w.window,
+            "kv_dtype": w.kv_dtype, "seed": w.seed}
+
+
+def main():
+    a = parse()
+    world, rank, local = dist_setup(a)
+    w = W.make_workload(a.config)
+    if a.impl == "reference":
+        run_reference(a, w)
+        return
+    import token_level_sparse_hs2_b200 as hs2
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    d = W.to_device(w, dev)
+    cache = hs2.KvCache(d["k"], d["v"], w.kv_start, w.kv_len, w.n_q, w.n_heads,
+                        d["k_scale"], d["v_scale"])
+    R, H, L = w.n_rows, w.n_heads, w.n_sparse
+    stride = int(w.kv_len.max())
+    cap = min(stride, w.topk + w.window)
+    out = torch.empty((w.batch, w.n_q, H, 128), dtype=torch.bfloat16, device=dev)
+    outs = [torch.empty_like(out) for _ in range(L)]
+    lse = torch.empty((w.batch, w.n_q, H), dtype=torch.float32, device=dev)
+    scores = torch.empty((R, stride), dtype=torch.float32, device=dev)
+    idx = torch.empty((R, cap), dtype=torch.int32, device=dev)
+    cnt = torch.empty(R, dtype=torch.int32, device=dev)
+    ws = torch.empty(hs2.workspace_size(cache, w.topk, w.window), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        hs2.block_decode(cache, d["q_full"], d["q_sparse"], out, outs, lse, scores, idx, cnt, ws,
+                         topk=w.topk, window=w.window)
+
+    for _ in range(a.warmup):
+        step()
+    hs2.read_device_status(ws)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    # ---- timed region: K steps, per-step events around every kernel
+    n_ev = 5 + L
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(a.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for row in evs:            # torch creates the CUDA event on first record
+        for e in row:
+            e.record(stream)
+    barrier()
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for k in range(a.steps):
+            hs2.block_decode_traced(cache, d["q_full"], d["q_sparse"], out, outs, lse, scores,
+                                    idx, cnt, ws, evs[k], topk=w.topk, window=w.window)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    hs2.read_device_status(ws)
+    ms = t_start.elapsed_time(t_end) / a.steps
+    ms_t = torch.tensor([ms], device=dev)
+    if pg:
+        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    names = ["clear", "pass1", "pass2", "topk"] + [f"sparse{l}" for l in range(L)]
+    per = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(a.steps))
+           for i, n in enumerate(names)}
+
+    # ---- same steps without per-kernel events (checks the tracing costs nothing)
+    barrier()
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0e.record(stream)
+    for _ in range(a.steps):
+        step()
+    t1e.record(stream)
+    torch.cuda.synchronize()
+    ms_plain = t0e.elapsed_time(t1e) / a.steps
+
+    # ---- end to end through the public API: host queries in, host results out, every step
+    e2e = None
+    if not a.no_e2e:
+        hq = d["q_full"].cpu().pin_memory()
+        hqs = [q.cpu().pin_memory() for q in d["q_sparse"]]
+        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hos = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(L)]
+        hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+        hcnt = torch.empty(cnt.shape, dtype=cnt.dtype).pin_memory()
+        dq = torch.empty_like(d["q_full"])
+        dqs = [torch.empty_like(q) for q in d["q_sparse"]]
+        h2d = hq.numel() * 2 + sum(q.numel() * 2 for q in hqs)
+        d2h = ho.numel() * 2 * (1 + L) + hidx.numel() * 4 + hcnt.numel() * 4
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            for x, y in zip(dqs, hqs):
+                x.copy_(y, non_blocking=True)
+            hs2.block_decode(cache, dq, dqs, out, outs, lse, scores, idx, cnt, ws,
+                             topk=w.topk, window=w.window)
+            ho.copy_(out, non_blocking=True)
+            for x, y in zip(hos, outs):
+                x.copy_(y, non_blocking=True)
+            hidx.copy_(idx, non_blocking=True)
+            hcnt.copy_(cnt, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(a.steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = torch.tensor([a0.elapsed_time(a1) / a.steps], device=dev)
+        if pg:
+            pg.all_reduce(ems, op=pg.ReduceOp.MAX)
+        e2e = {"value": world * R / (float(ems.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": float(ems.item())}
+
+    hbm, how = peaks()
+    ab = algorithmic_bytes(w)
+    p1_s = per["pass1"] / 1e3
+    ach = ab["pass1"] / p1_s / 1e9
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            traffic = json.load(f).get(w.name, {}).get("pass1")
+    except Exception:
+        pass
+    kernels_per_step = 2 + 1 + L   # pass 1, pass 2, selection, sparse layers
+    line = {
+        "metric": METRIC, "value": world * R / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.kv_dtype == "bf16" else "fp8-e4m3 (bf16/f16 math)",
+        "data": "synthetic",
+        "config": dict(config_of(w), parallelism=f"replicas x{world} (independent batches)",
+                       l2="inputs larger than L2 (K/V cache %.0f MB > 126 MB); no flush"
+                          % (w.k.nbytes * 2 / 1e6)),
+        "roofline": {"kernel": "full-attention pass 1", "bound": "hbm", "achieved": ach,
+                     "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": traffic,
+                     "peak_source": how, "bytes_per_launch": ab["pass1"],
+                     "ms_per_launch": per["pass1"]},
+        "block_roofline": {"bytes_per_step": ab["total"],
+                           "achieved_gbs": ab["total"] / (ms_max / 1e3) / 1e9,
+                           "frac": ab["total"] / (ms_max / 1e3) / 1e9 / hbm},
+        "ms_per_kernel": per, "ms_per_step_untraced": ms_plain,
+        "gpu_launches": kernels_per_step * a.steps,
+        "clocks": clk.result(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

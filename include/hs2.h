@@ -1,0 +1,171 @@
+/*
+ * hs2.h -- C ABI of libhs2: the KV-Reuse token-sparse attention of one HySparse2 hybrid block
+ * on an NVIDIA B200 (sm_100a).
+ *
+ * The operation (HySparse2 pages):
+ *  - "HySparse2: How Xiaomi Split the Transformer to Fix Agent Prefill Costs", section
+ *    "KV Reuse and Token-Level Sparse Selection": a hybrid block of the cross-decoder is one
+ *    full-attention layer followed by sparse-attention layers. The full layer attends over the
+ *    whole context and produces both the KV cache and token selection indices; the sparse
+ *    layers reuse the indices and the cache without recomputing them. Selection is per token:
+ *    1,024 tokens from the whole context plus a forced window of the 128 most recent tokens,
+ *    read from the full layer's cache.
+ *  - "HySparse2: Hybrid Sparse Attention with Two-Level KV Sharing", bullets "KV Reuse
+ *    refinements" and "Inference cost": token-level selection, forced local window, MQA (one
+ *    K/V head for all query heads), FP8 KV cache.
+ * Readings where the pages are silent: the importance score of cache position t for a query
+ * row is s[t] = sum_h exp(c * q_h . k_t - lse_h), c = softmax_scale (1/sqrt(128) by default),
+ * computed in a second pass from the full layer's log-sum-exp; ties go to the lower index;
+ * the window is not part of the candidate set; the selected set is returned ascending.
+ *
+ * Conventions for every call:
+ *  - Device pointers are CUDA global-memory pointers on the current device; "HOST" marks the
+ *    few host pointers. The caller owns every buffer. The library allocates nothing, keeps no
+ *    state between calls, and launches only on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream). Calls return after enqueueing; nothing synchronises.
+ *  - Argument errors are detected on the host before anything is enqueued and returned as
+ *    HS2_ERR_INVALID_ARG / HS2_ERR_UNSUPPORTED / HS2_ERR_WORKSPACE with a message in
+ *    hs2_last_error(). A CUDA launch error returns HS2_ERR_CUDA. Errors found by the kernels
+ *    themselves (a bounded wait that ran out) are recorded in the workspace and read back with
+ *    hs2_read_device_status(). No C++ exception crosses this interface.
+ *  - Shapes: B = batch, Nq = query tokens per sequence (1 for decode), H = query heads,
+ *    d = 128. Query i of sequence b sits at cache position p = T_b - Nq + i and attends
+ *    causally to positions [0, p] of its own sequence. Flat query row r = b * Nq + i.
+ *  - Calls that overlap on the GPU must not share a workspace.
+ */
+#ifndef HS2_H_
+#define HS2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HS2_VERSION 1
+#define HS2_HEAD_DIM 128
+#define HS2_MAX_BATCH 128     /* sequences per call */
+#define HS2_MAX_TOPK 2048     /* global selection budget per query row */
+#define HS2_MAX_WINDOW 4096   /* forced recent window per query row */
+
+typedef enum {
+  HS2_OK = 0,
+  HS2_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad shape, inconsistent sizes */
+  HS2_ERR_UNSUPPORTED = 2,   /* valid but not implemented: head_dim != 128, H not 16/32, ... */
+  HS2_ERR_WORKSPACE = 3,     /* workspace smaller than hs2_workspace_size() */
+  HS2_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  HS2_ERR_DEVICE_CHECK = 5,  /* a kernel's own consistency check failed (device status) */
+  HS2_ERR_TIMEOUT = 6        /* a kernel's bounded wait ran out (device status) */
+} hs2_status;
+
+typedef enum {
+  HS2_KV_BF16 = 0,           /* K, V rows of 128 bf16 */
+  HS2_KV_FP8_E4M3 = 1        /* K, V rows of 128 OCP e4m3fn codes; value = scale[row] * code */
+} hs2_kv_dtype;
+
+typedef enum { HS2_OUT_BF16 = 0, HS2_OUT_F32 = 1 } hs2_out_dtype;
+
+/* The shared single-head (MQA) K/V cache of one full-attention layer, and the query shape.
+ * Sequence b occupies cache rows [kv_start[b], kv_start[b] + kv_len[b]); its queries are its
+ * last n_q tokens. Row-major [kv_rows, 128]; each row is one token's K (or V). */
+typedef struct hs2_kv_view {
+  int32_t batch;             /* B, 1..HS2_MAX_BATCH */
+  int32_t n_q;               /* Nq >= 1; every kv_len[b] >= n_q */
+  int32_t n_heads;           /* H: 16 or 32 query heads share the one K/V head */
+  int32_t head_dim;          /* must be 128 */
+  int32_t kv_dtype;          /* hs2_kv_dtype */
+  int32_t reserved;          /* must be 0 */
+  int64_t kv_rows;           /* rows of k / v / k_scale / v_scale (>= every sequence's end) */
+  const void *k;             /* device, 16-byte aligned */
+  const void *v;             /* device, 16-byte aligned */
+  const float *k_scale;      /* device [kv_rows], 16-byte aligned, FP8 only (else NULL) */
+  const float *v_scale;      /* device [kv_rows], 16-byte aligned, FP8 only (else NULL) */
+  const int64_t *kv_start;   /* HOST [batch] */
+  const int32_t *kv_len;     /* HOST [batch], T_b */
+} hs2_kv_view;
+
+/* Bytes of device scratch the calls below need for this view and budget (same value for every
+ * call on the view). Any 256-byte-aligned device buffer of at least this size works; its
+ * contents on entry do not matter. Host-only; does not touch the GPU. */
+hs2_status hs2_workspace_size(const hs2_kv_view *kv, int32_t topk, int32_t window,
+                              size_t *bytes);
+
+/* Step 1 -- the full-attention layer and its importance scores (pages: section "KV Reuse and
+ * Token-Level Sparse Selection"; the full layer attends causally over the entire context).
+ * For every query row r and head h:
+ *   lse[r,h]  = log sum_{t<=p} exp(c q_h.k_t)
+ *   out[r,h,:] = sum_{t<=p} exp(c q_h.k_t - lse[r,h]) v_t
+ *   scores[r * score_stride + t] = sum_h exp(c q_h.k_t - lse[r,h])      for t in [0, p]
+ * q: device bf16 [B, Nq, H, 128]. out: device [B, Nq, H, 128] of out_dtype. lse: device fp32
+ * [B, Nq, H]. scores: device fp32, score_stride >= max p + 1 (entries past p are not written).
+ * The scores are written by a second pass over K that uses the final lse. */
+hs2_status hs2_full_attn_scores(const hs2_kv_view *kv, const void *q, float softmax_scale,
+                                void *out, int32_t out_dtype, float *lse, float *scores,
+                                int64_t score_stride, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/* Step 2 -- token-level top-k plus forced window (pages: "KV Reuse and Token-Level Sparse
+ * Selection"; "KV Reuse refinements"). For query row r at position p: candidates
+ * C = [0, nc) with nc = max(0, p - window + 1), window W = [nc, p]. If nc <= topk the selection
+ * is [0, p]; otherwise it is the topk candidates with the largest score (ties: lower index),
+ * followed by W, all ascending. Scores are compared by their fp32 bit patterns, which for the
+ * non-negative scores step 1 produces is the numeric order (an exact, deterministic radix
+ * select). idx: device int32 [B*Nq, idx_stride], idx_stride >= min(max p + 1, topk + window);
+ * only the first count[r] entries of row r are written. count: device int32 [B*Nq]. */
+hs2_status hs2_topk_select(const hs2_kv_view *kv, const float *scores, int64_t score_stride,
+                           int32_t topk, int32_t window, int32_t *idx, int32_t idx_stride,
+                           int32_t *count, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+/* Step 3 -- one sparse-attention layer with KV Reuse (pages: section "KV Reuse and Token-Level
+ * Sparse Selection"; sparse layers take the full layer's indices as they are, and window tokens
+ * come from the same cache the full layer wrote). Each query row
+ * attends only to its selected positions; each gathered K/V row is loaded once for all heads:
+ *   out[r,h,:] = sum_{j<count[r]} softmax_j(c q_h.k_{S_j}) v_{S_j},  S = idx[r, :count[r]]
+ * q: device bf16 [B, Nq, H, 128] (this layer's own queries). Indices must lie in [0, p];
+ * count[r] must be in [1, idx_stride] and at most topk + window of the workspace sizing. */
+hs2_status hs2_sparse_gather_attn(const hs2_kv_view *kv, const void *q, const int32_t *idx,
+                                  int32_t idx_stride, const int32_t *count,
+                                  float softmax_scale, void *out, int32_t out_dtype,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* The whole hybrid block: step 1, step 2, then n_sparse sparse layers that reuse the indices
+ * and the cache, enqueued back to back on `stream`. q_sparse / out_sparse are HOST arrays of
+ * n_sparse device pointers (layouts as in step 3). lse, scores, idx and count are outputs too
+ * (caller-provided, layouts as above). n_sparse may be 0. */
+hs2_status hs2_block_decode(const hs2_kv_view *kv, const void *q_full,
+                            const void *const *q_sparse, int32_t n_sparse, int32_t topk,
+                            int32_t window, float softmax_scale, void *out_full,
+                            void *const *out_sparse, int32_t out_dtype, float *lse,
+                            float *scores, int64_t score_stride, int32_t *idx,
+                            int32_t idx_stride, int32_t *count, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/* hs2_block_decode, plus one cudaEvent_t (cast to void *) recorded on `stream` before the
+ * first enqueued operation and after each step: events[0] before the workspace clear,
+ * events[1] after it, events[2] after full-attention pass 1, events[3] after score pass 2,
+ * events[4] after the selection, events[5 + l] after sparse layer l. n_events must be
+ * 5 + n_sparse. For timing individual kernels without a profiler; results are identical. */
+hs2_status hs2_block_decode_traced(const hs2_kv_view *kv, const void *q_full,
+                                   const void *const *q_sparse, int32_t n_sparse, int32_t topk,
+                                   int32_t window, float softmax_scale, void *out_full,
+                                   void *const *out_sparse, int32_t out_dtype, float *lse,
+                                   float *scores, int64_t score_stride, int32_t *idx,
+                                   int32_t idx_stride, int32_t *count, void *workspace,
+                                   size_t workspace_bytes, void *const *events,
+                                   int32_t n_events, void *stream);
+
+/* Synchronises `stream` and returns the status the kernels of the last call on this workspace
+ * recorded: HS2_OK, HS2_ERR_TIMEOUT or HS2_ERR_DEVICE_CHECK (HS2_ERR_CUDA if the read fails). */
+hs2_status hs2_read_device_status(const void *workspace, void *stream);
+
+/* Message for the last non-OK status returned on the calling thread ("" if none). */
+const char *hs2_last_error(void);
+const char *hs2_status_string(hs2_status status);
+int32_t hs2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HS2_H_ */

@@ -1,0 +1,158 @@
+"""The C ABI on the CPU: the library loads, exports every entry point include/hs2.h declares,
+and rejects bad arguments on the host before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import token_level_sparse_hs2_b200 as hs2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from token_level_sparse_hs2_b200 import build
+    build.build()
+    return hs2.lib()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(hs2_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert {"hs2_block_decode", "hs2_full_attn_scores", "hs2_topk_select",
+            "hs2_sparse_gather_attn", "hs2_workspace_size"} <= names
+    for n in sorted(names):
+        assert hasattr(L, n), n
+    assert L.hs2_version() == 1
+    assert L.hs2_status_string(6) == b"HS2_ERR_TIMEOUT"
+
+
+def cpu_cache(batch=2, n_q=1, H=32, d=128, lens=(300, 500), dtype=torch.bfloat16, **kw):
+    rows = sum(lens) + 8
+    k = torch.zeros((rows, d), dtype=dtype)
+    v = torch.zeros((rows, d), dtype=dtype)
+    start = [0]
+    for t in lens[:-1]:
+        start.append(start[-1] + t)
+    ks = vs = None
+    if dtype == torch.uint8:
+        ks = torch.ones(rows)
+        vs = torch.ones(rows)
+    c = hs2.KvCache(k, v, start, lens, n_q, H, ks, vs)
+    c.view.head_dim = d
+    for key, val in kw.items():
+        setattr(c.view, key, val)
+    return c
+
+
+def status_of(fn):
+    try:
+        fn()
+    except hs2.HS2Error as e:
+        return e.status, str(e)
+    return 0, ""
+
+
+def test_workspace_size_host_only(L):
+    c = cpu_cache()
+    n = hs2.workspace_size(c)
+    assert n > 0 and n % 256 == 0
+    assert hs2.workspace_size(cpu_cache(lens=(300, 5000))) >= n
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(head_dim=64), 2),
+    (dict(n_heads=8), 2),
+    (dict(batch=0), 1),
+    (dict(n_q=0), 1),
+    (dict(kv_dtype=7), 1),
+    (dict(reserved=1), 1),
+    (dict(kv_rows=10), 1),
+])
+def test_view_validation(L, kw, expect):
+    c = cpu_cache()
+    for key, val in kw.items():
+        setattr(c.view, key, val)
+    st, msg = status_of(lambda: hs2.workspace_size(c))
+    assert st == expect, msg
+
+
+def test_misaligned_and_null_pointers(L):
+    c = cpu_cache()
+    c.view.k = c.view.k + 2
+    assert status_of(lambda: hs2.workspace_size(c))[0] == 1
+    c = cpu_cache()
+    c.view.v = None
+    assert status_of(lambda: hs2.workspace_size(c))[0] == 1
+    c = cpu_cache(dtype=torch.uint8)
+    c.view.k_scale = None
+    assert status_of(lambda: hs2.workspace_size(c))[0] == 1
+
+
+def test_sequence_shorter_than_queries(L):
+    c = cpu_cache(n_q=400)
+    st, msg = status_of(lambda: hs2.workspace_size(c))
+    assert st == 1 and "n_q" in msg
+
+
+def test_budget_limits(L):
+    c = cpu_cache()
+    assert status_of(lambda: hs2.workspace_size(c, topk=0))[0] == 2
+    assert status_of(lambda: hs2.workspace_size(c, topk=4096))[0] == 2
+    assert status_of(lambda: hs2.workspace_size(c, window=-1))[0] == 2
+
+
+def test_call_argument_checks_before_any_launch(L):
+    c = cpu_cache()
+    H = 32
+    q = torch.zeros((2, 1, H, 128), dtype=torch.bfloat16)
+    out = torch.zeros_like(q, dtype=torch.float32)
+    lse = torch.zeros((2, 1, H))
+    scores = torch.zeros((2, 500))
+    idx = torch.zeros((2, 500), dtype=torch.int32)
+    cnt = torch.zeros(2, dtype=torch.int32)
+    def aligned(n):
+        buf = torch.zeros(n + 256, dtype=torch.uint8)
+        off = (-buf.data_ptr()) % 256
+        return buf, buf.data_ptr() + off
+    ws_buf, ws_ptr = aligned(hs2.workspace_size(c))
+    small_buf, small_ptr = aligned(256)
+    raw = hs2.lib().hs2_block_decode
+    args = lambda **o: [o.get("view", c.ref()), q.data_ptr(),
+                        (ctypes.c_void_p * 1)(q.data_ptr()), o.get("n_sparse", 1), 1024, 128,
+                        o.get("scale", 0.088), out.data_ptr(),
+                        (ctypes.c_void_p * 1)(out.data_ptr()), 1, lse.data_ptr(),
+                        scores.data_ptr(), o.get("score_stride", 500), idx.data_ptr(),
+                        o.get("idx_stride", 500), cnt.data_ptr(), o.get("ws", ws_ptr),
+                        o.get("ws_bytes", ws_buf.numel() - 256), None]
+    st = raw(*args(ws=small_ptr, ws_bytes=256))
+    assert st == 3, hs2.lib().hs2_last_error()
+    assert raw(*args(score_stride=499)) == 1
+    assert raw(*args(idx_stride=100)) == 1
+    assert raw(*args(scale=float("nan"))) == 1
+    assert raw(*args(scale=0.0)) == 1
+    assert raw(*args(n_sparse=-1)) == 1
+    assert raw(*args(ws=ws_ptr + 16)) == 1
+    st = raw(*args(score_stride=499))
+    assert st == 1 and b"score_stride" in hs2.lib().hs2_last_error()
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    import importlib
+    mod = importlib.import_module("token_level_sparse_hs2_b200")
+    monkeypatch.setattr(mod, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(mod, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        mod.lib()

@@ -1,0 +1,164 @@
+"""GPU parity for the decode hybrid block (one query token per sequence), through the C ABI,
+against the fp64 oracle on the same seeded inputs. Tolerances are in tests/gpu_helpers.py."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from token_level_sparse_hs2_b200 import build
+    build.build()
+    oracle.build()
+
+
+def H():
+    from tests import gpu_helpers
+    return gpu_helpers
+
+
+def decode(**kw):
+    cfg = dict(name="decode_small", batch=1, n_q=1, n_heads=32, n_sparse=2, kv_dtype="bf16",
+               lengths=(4096,), needles=8)
+    cfg.update(kw)
+    return W.make_workload(cfg, seed=kw.pop("seed", 17))
+
+
+def test_config0_decode_4k():
+    w = W.make_workload(0)
+    g = H().run_block(w)
+    H().check_block(w, g)
+    sel = set(g["idx"][0, :g["count"][0]].tolist())
+    assert set(w.needle_pos[0].tolist()) <= sel
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("heads", [16, 32])
+def test_ragged_batch(kv_dtype, heads):
+    # several tiles per sequence, ragged tails, tile boundaries shared by two sequences
+    w = decode(batch=3, lengths=(3000, 1500, 2701), n_heads=heads, kv_dtype=kv_dtype, needles=5)
+    g = H().run_block(w)
+    H().check_block(w, g)
+
+
+def test_short_contexts_keep_everything():
+    lens = (1, 2, 127, 128, 129, 1151, 1152, 1153)
+    w = decode(batch=len(lens), lengths=lens, n_heads=16, needles=0)
+    g = H().run_block(w)
+    H().check_block(w, g)
+    for b, T in enumerate(lens):
+        assert g["count"][b] == min(T, 1152)
+        if T <= 1152:
+            assert np.array_equal(g["idx"][b, :T], np.arange(T))
+
+
+@pytest.mark.parametrize("topk,window", [(8, 4), (3, 1), (64, 0), (2048, 256)])
+def test_budget_variants(topk, window):
+    w = decode(batch=2, lengths=(700, 3000), topk=topk, window=window, needles=2)
+    g = H().run_block(w)
+    H().check_block(w, g)
+
+
+def test_bf16_outputs():
+    w = decode(batch=2, lengths=(2000, 900))
+    g = H().run_block(w, out_dtype=torch.bfloat16)
+    H().check_block(w, g)
+
+
+def test_workspace_contents_do_not_matter():
+    w = decode(batch=2, lengths=(20000, 5000))
+    g = H().run_block(w, ws_fill=0xFF)
+    H().check_block(w, g)
+
+
+def test_deterministic():
+    w = decode(batch=2, lengths=(40000, 9000), kv_dtype="fp8")
+    a = H().run_block(w)
+    b = H().run_block(w)
+    for key in ("o_full", "lse", "idx", "count"):
+        assert np.array_equal(a[key], b[key]), key
+    assert np.array_equal(np.nan_to_num(a["scores"], nan=-1), np.nan_to_num(b["scores"], nan=-1))
+    for x, y in zip(a["o_sparse"], b["o_sparse"]):
+        assert np.array_equal(x, y)
+
+
+def test_all_scores_equal_takes_lowest_indices():
+    # identical keys: every score is H/(p+1); the compacted set overflows and the exact
+    # fallback must pick [0, topk) plus the window
+    w = decode(batch=1, lengths=(20000,), needles=0)
+    w.k = np.tile(w.k[:1], (w.kv_rows, 1))
+    g = H().run_block(w)
+    p = 19999
+    nc = p - 127
+    assert np.array_equal(g["idx"][0, :1152], np.concatenate([np.arange(1024), np.arange(nc, p + 1)]))
+    H().check_block(w, g)
+
+
+def test_topk_standalone_matches_block():
+    import token_level_sparse_hs2_b200 as hs2
+    w = decode(batch=2, lengths=(50000, 3000))
+    g = H().run_block(w)
+    dev = torch.device("cuda")
+    scores = torch.from_numpy(g["scores"]).to(dev)
+    idx = torch.full_like(torch.from_numpy(g["idx"]), -1).to(dev)
+    cnt = torch.zeros(w.n_rows, dtype=torch.int32, device=dev)
+    hs2.topk_select(g["cache"], scores, idx, cnt, g["ws"])
+    hs2.read_device_status(g["ws"])
+    assert np.array_equal(cnt.cpu().numpy(), g["count"])
+    for r in range(w.n_rows):
+        c = g["count"][r]
+        assert np.array_equal(idx[r, :c].cpu().numpy(), g["idx"][r, :c])
+
+
+@pytest.mark.parametrize("n,quant", [(100000, 0), (100000, 64), (30000, 4), (5000, 0)])
+def test_topk_on_synthetic_scores(n, quant):
+    """Integer work is bit-exact: arbitrary non-negative scores (heavy ties when quantised,
+    denormals and zeros included) against the oracle's fp32 selector."""
+    import token_level_sparse_hs2_b200 as hs2
+    rng = np.random.default_rng(n + quant)
+    lens = (n, n // 2 + 3)
+    w = decode(batch=2, lengths=lens, needles=0)
+    s = rng.lognormal(0, 2, size=(2, n)).astype(np.float32)
+    if quant:
+        s = (np.round(s * quant) / quant).astype(np.float32)
+    s[:, :50] = np.array([0.0, 1e-45, 3e-39] * 17, dtype=np.float32)[:50]
+    d = W.to_device(w)
+    cache = hs2.KvCache(d["k"], d["v"], w.kv_start, w.kv_len, 1, w.n_heads)
+    dev = torch.device("cuda")
+    scores = torch.from_numpy(s).to(dev)
+    idx = torch.full((2, 1152), -1, dtype=torch.int32, device=dev)
+    cnt = torch.zeros(2, dtype=torch.int32, device=dev)
+    ws = torch.empty(hs2.workspace_size(cache), dtype=torch.uint8, device=dev)
+    hs2.topk_select(cache, scores, idx, cnt, ws)
+    hs2.read_device_status(ws)
+    ref, rc = oracle.select_rows(w, np.arange(2), s, fp32=True)
+    got, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+    for r in range(2):
+        assert gc[r] == rc[r]
+        assert np.array_equal(got[r, :gc[r]], ref[r, :rc[r]])
+
+
+@pytest.mark.slow
+def test_config1_full_size():
+    w = W.make_workload(1)
+    g = H().run_block(w)
+    H().check_block(w, g)
+    for b in range(w.batch):
+        sel = set(g["idx"][b, :g["count"][b]].tolist())
+        assert set(w.needle_pos[b].tolist()) <= sel
+
+
+@pytest.mark.slow
+def test_config2_full_size_fp8():
+    w = W.make_workload(2)
+    g = H().run_block(w)
+    H().check_block(w, g)
+    sel = set(g["idx"][0, :g["count"][0]].tolist())
+    assert set(w.needle_pos[0].tolist()) <= sel

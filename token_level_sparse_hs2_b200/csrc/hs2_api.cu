@@ -1,0 +1,572 @@
+// hs2_api.cu -- the C ABI of libhs2 (declared in include/hs2.h): argument validation on the
+// host, the work plan (how each step is split over CTAs), workspace carving, TMA descriptors
+// and the launch sequence of one hybrid block:
+//   full-attention pass 1 -> score pass 2 -> top-k + window -> sparse layer x n_sparse.
+// Nothing here allocates, synchronises or keeps state between calls.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <functional>
+#include <mutex>
+
+#include "internal.h"
+
+namespace hs2 {
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+hs2_status fail(hs2_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+hs2_status ok() {
+  g_err[0] = '\0';
+  return HS2_OK;
+}
+
+constexpr int kTargetItems = 4 * 148;     // decode work items per pass (~4 per SM)
+constexpr int kSegLen = 16384;            // top-k candidates per CTA when rows are split
+constexpr int kManyRows = 148;            // rows at least this many: one CTA per row
+constexpr int kCandCapGlobal = 8192;
+constexpr int kMaxSplit = 32;             // sparse-layer CTAs per query row, at most
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Work plan and workspace layout for one view.
+struct Plan {
+  int B = 0, n_q = 0, H = 0, kv_dtype = 0;
+  int64_t kv_rows = 0, max_p = 0;
+  int n_rows = 0;
+  // decode passes
+  int chunk_tiles = 1, n_items = 0;
+  int32_t item_begin[HS2_MAX_BATCH + 1] = {};
+  // top-k
+  int n_seg = 1, seg_len = 0;
+  // sparse layers: n_split chosen per call from the index capacity
+  bool sparse_split = false;
+  // workspace (byte offsets); [0, zero_end) is cleared at the start of every call
+  size_t off_status = 0, off_cnt_p1 = 0, off_hist = 0, off_cand_count = 0, off_arrive = 0,
+         off_cnt_sp = 0, zero_end = 0;
+  size_t off_part_p1 = 0, off_cand_key = 0, off_cand_idx = 0, off_part_sp = 0, total = 0;
+};
+
+hs2_status validate_view(const hs2_kv_view *kv) {
+  if (!kv) return fail(HS2_ERR_INVALID_ARG, "kv view is NULL");
+  if (kv->batch < 1 || kv->batch > HS2_MAX_BATCH)
+    return fail(HS2_ERR_INVALID_ARG, "batch %d outside [1, %d]", kv->batch, HS2_MAX_BATCH);
+  if (kv->n_q < 1) return fail(HS2_ERR_INVALID_ARG, "n_q %d < 1", kv->n_q);
+  if (kv->head_dim != HS2_HEAD_DIM)
+    return fail(HS2_ERR_UNSUPPORTED, "head_dim %d (only 128 is supported)", kv->head_dim);
+  if (kv->n_heads != 16 && kv->n_heads != 32)
+    return fail(HS2_ERR_UNSUPPORTED, "n_heads %d (16 or 32 query heads per K/V head)", kv->n_heads);
+  if (kv->kv_dtype != HS2_KV_BF16 && kv->kv_dtype != HS2_KV_FP8_E4M3)
+    return fail(HS2_ERR_INVALID_ARG, "kv_dtype %d", kv->kv_dtype);
+  if (kv->reserved != 0) return fail(HS2_ERR_INVALID_ARG, "reserved field must be 0");
+  if (kv->kv_rows < 1 || kv->kv_rows > (int64_t)INT32_MAX - 2 * 64)
+    return fail(HS2_ERR_INVALID_ARG, "kv_rows %lld out of range", (long long)kv->kv_rows);
+  if (!kv->k || !kv->v) return fail(HS2_ERR_INVALID_ARG, "k / v is NULL");
+  if (!aligned16(kv->k) || !aligned16(kv->v))
+    return fail(HS2_ERR_INVALID_ARG, "k / v must be 16-byte aligned");
+  if (kv->kv_dtype == HS2_KV_FP8_E4M3) {
+    if (!kv->k_scale || !kv->v_scale)
+      return fail(HS2_ERR_INVALID_ARG, "FP8 cache needs k_scale and v_scale");
+    if (!aligned16(kv->k_scale) || !aligned16(kv->v_scale))
+      return fail(HS2_ERR_INVALID_ARG, "k_scale / v_scale must be 16-byte aligned");
+  }
+  if (!kv->kv_start || !kv->kv_len) return fail(HS2_ERR_INVALID_ARG, "kv_start / kv_len is NULL");
+  for (int b = 0; b < kv->batch; ++b) {
+    const int64_t s = kv->kv_start[b];
+    const int32_t T = kv->kv_len[b];
+    if (T < kv->n_q)
+      return fail(HS2_ERR_INVALID_ARG, "kv_len[%d] = %d < n_q = %d", b, T, kv->n_q);
+    if (s < 0 || s + T > kv->kv_rows)
+      return fail(HS2_ERR_INVALID_ARG, "sequence %d rows [%lld, %lld) outside [0, %lld)", b,
+                  (long long)s, (long long)(s + T), (long long)kv->kv_rows);
+  }
+  return HS2_OK;
+}
+
+void make_plan(const hs2_kv_view *kv, Plan &P) {
+  P.B = kv->batch;
+  P.n_q = kv->n_q;
+  P.H = kv->n_heads;
+  P.kv_dtype = kv->kv_dtype;
+  P.kv_rows = kv->kv_rows;
+  P.n_rows = P.B * P.n_q;
+  P.max_p = 0;
+  int64_t total_tiles = 0;
+  for (int b = 0; b < P.B; ++b) {
+    P.max_p = std::max<int64_t>(P.max_p, kv->kv_len[b] - 1);
+    const int64_t r0 = kv->kv_start[b], r1 = r0 + kv->kv_len[b];
+    total_tiles += (r1 + kTile - 1) / kTile - r0 / kTile;
+  }
+  // decode items: chunks of chunk_tiles tiles per sequence
+  P.chunk_tiles = (int)std::max<int64_t>(1, (total_tiles + kTargetItems - 1) / kTargetItems);
+  P.n_items = 0;
+  for (int b = 0; b < P.B; ++b) {
+    const int64_t r0 = kv->kv_start[b], r1 = r0 + kv->kv_len[b];
+    const int64_t tiles = (r1 + kTile - 1) / kTile - r0 / kTile;
+    P.item_begin[b] = P.n_items;
+    P.n_items += (int)((tiles + P.chunk_tiles - 1) / P.chunk_tiles);
+  }
+  P.item_begin[P.B] = P.n_items;
+  // top-k segments: split long rows when there are few of them
+  const int64_t max_cand = P.max_p + 1;
+  if (P.n_rows >= kManyRows) {
+    P.n_seg = 1;
+  } else {
+    P.n_seg = (int)std::min<int64_t>(256, std::max<int64_t>(1, (max_cand + kSegLen - 1) / kSegLen));
+  }
+  P.seg_len = (int)((max_cand + P.n_seg - 1) / P.n_seg);
+  P.sparse_split = P.n_rows < 2 * kManyRows;
+
+  // workspace layout
+  size_t o = 0;
+  P.off_status = o; o = align_up(o + 4);
+  P.off_cnt_p1 = o; o = align_up(o + 4 * (size_t)P.B);
+  P.off_hist = o; o = align_up(o + (P.n_seg > 1 ? 4 * (size_t)kHistBins * P.n_rows : 0));
+  P.off_cand_count = o; o = align_up(o + 4 * (size_t)P.n_rows);
+  P.off_arrive = o; o = align_up(o + 4 * (size_t)P.n_rows);
+  P.off_cnt_sp = o; o = align_up(o + 4 * (size_t)P.n_rows);
+  P.zero_end = o;
+  const size_t part_row = (size_t)P.H * (2 + kHeadDim) * 4;
+  P.off_part_p1 = o; o = align_up(o + (P.n_q == 1 ? part_row * P.n_items : 0));
+  const size_t cand = (P.n_seg > 1) ? (size_t)P.n_rows * kCandCapGlobal * 4 : 0;
+  P.off_cand_key = o; o = align_up(o + cand);
+  P.off_cand_idx = o; o = align_up(o + cand);
+  P.off_part_sp = o; o = align_up(o + (P.sparse_split ? part_row * kMaxSplit * P.n_rows : 0));
+  P.total = o;
+}
+
+void fill_seq(const hs2_kv_view *kv, const Plan &P, SeqTable &t) {
+  memset(&t, 0, sizeof t);
+  for (int b = 0; b < P.B; ++b) {
+    t.start[b] = kv->kv_start[b];
+    t.len[b] = kv->kv_len[b];
+    t.item_begin[b] = P.item_begin[b];
+  }
+  t.item_begin[P.B] = P.item_begin[P.B];
+}
+
+hs2_status check_ws(const Plan &P, void *ws, size_t bytes) {
+  if (!ws) return fail(HS2_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign)
+    return fail(HS2_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (bytes < P.total)
+    return fail(HS2_ERR_WORKSPACE, "workspace %zu bytes < %zu required", bytes, P.total);
+  return HS2_OK;
+}
+
+template <class T>
+T *ws_at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+hs2_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  return HS2_OK;
+}
+
+hs2_status encode_maps(const hs2_kv_view *kv, TensorMaps &tm) {
+  hs2_status st = get_encoder();
+  if (st != HS2_OK) return st;
+  memset(&tm, 0, sizeof tm);
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r;
+  if (kv->kv_dtype == HS2_KV_BF16) {
+    const cuuint64_t dims[2] = {128, (cuuint64_t)kv->kv_rows};
+    const cuuint64_t strides[1] = {256};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+    for (int which = 0; which < 2; ++which) {
+      r = g_encode(which ? &tm.v : &tm.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void *>(which ? kv->v : kv->k), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled(K/V bf16) = %d", (int)r);
+    }
+  } else {
+    const cuuint64_t dims[2] = {128, (cuuint64_t)kv->kv_rows};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, (cuuint32_t)kTile};
+    for (int which = 0; which < 2; ++which) {
+      r = g_encode(which ? &tm.v : &tm.k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                   const_cast<void *>(which ? kv->v : kv->k), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled(K/V e4m3) = %d", (int)r);
+    }
+  }
+  return HS2_OK;
+}
+
+hs2_status cuda_check(cudaError_t e, const char *what) {
+  if (e != cudaSuccess) return fail(HS2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return HS2_OK;
+}
+
+bool valid_scale(float s) { return std::isfinite(s) && s > 0.f; }
+
+// ------------------------------------------------------------------ steps
+
+hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, const void *q,
+                    float scale, void *out, int out_f32, float *lse, float *scores,
+                    int64_t score_stride, int window, bool with_hist, void *ws,
+                    cudaStream_t stream, const std::function<hs2_status()> *mark = nullptr) {
+  if (P.n_q != 1)
+    return fail(HS2_ERR_UNSUPPORTED, "multi-token query chunks (n_q > 1) are not built yet");
+  DecodeParams dp;
+  memset(&dp, 0, sizeof dp);
+  fill_seq(kv, P, dp.seq);
+  dp.batch = P.B;
+  dp.n_heads = P.H;
+  dp.chunk_tiles = P.chunk_tiles;
+  dp.n_items = P.n_items;
+  dp.window = window;
+  dp.scale_log2 = scale * 1.4426950408889634f;
+  dp.kv_rows = kv->kv_rows;
+  dp.k_scale = kv->k_scale;
+  dp.v_scale = kv->v_scale;
+  dp.q = q;
+  dp.out = out;
+  dp.out_f32 = out_f32;
+  dp.lse = lse;
+  dp.scores = scores;
+  dp.score_stride = score_stride;
+  dp.hist = with_hist ? ws_at<uint32_t>(ws, P.off_hist) : nullptr;
+  dp.part = ws_at<float>(ws, P.off_part_p1);
+  dp.counter = ws_at<int32_t>(ws, P.off_cnt_p1);
+  dp.status = ws_at<uint32_t>(ws, P.off_status);
+  hs2_status st = cuda_check(launch_decode_pass(0, P.kv_dtype, tm, dp, stream), "full-attention pass 1");
+  if (st != HS2_OK) return st;
+  if (mark && (st = (*mark)()) != HS2_OK) return st;
+  st = cuda_check(launch_decode_pass(1, P.kv_dtype, tm, dp, stream), "score pass 2");
+  if (st != HS2_OK) return st;
+  if (mark && (st = (*mark)()) != HS2_OK) return st;
+  return HS2_OK;
+}
+
+hs2_status run_topk(const hs2_kv_view *kv, const Plan &P, const float *scores,
+                    int64_t score_stride, int topk, int window, int32_t *idx, int idx_stride,
+                    int32_t *count, bool hist_ready, void *ws, cudaStream_t stream) {
+  TopkParams tp;
+  memset(&tp, 0, sizeof tp);
+  fill_seq(kv, P, tp.seq);
+  tp.batch = P.B;
+  tp.n_q = P.n_q;
+  tp.topk = topk;
+  tp.window = window;
+  tp.scores = scores;
+  tp.score_stride = score_stride;
+  tp.n_seg = P.n_seg;
+  tp.seg_len = P.seg_len;
+  if (P.n_seg > 1) {
+    if (hist_ready) tp.hist = ws_at<uint32_t>(ws, P.off_hist);
+    else tp.hist_ws = ws_at<uint32_t>(ws, P.off_hist);
+  }
+  tp.cand_key = ws_at<uint32_t>(ws, P.off_cand_key);
+  tp.cand_idx = ws_at<int32_t>(ws, P.off_cand_idx);
+  tp.cand_cap = kCandCapGlobal;
+  tp.cand_count = ws_at<int32_t>(ws, P.off_cand_count);
+  tp.arrive = ws_at<int32_t>(ws, P.off_arrive);
+  tp.idx = idx;
+  tp.idx_stride = idx_stride;
+  tp.count = count;
+  tp.status = ws_at<uint32_t>(ws, P.off_status);
+  return cuda_check(launch_topk(tp, P.n_rows, stream), "top-k selection");
+}
+
+hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const int32_t *idx,
+                      int idx_stride, const int32_t *count, float scale, void *out, int out_f32,
+                      void *ws, cudaStream_t stream) {
+  SparseParams sp;
+  memset(&sp, 0, sizeof sp);
+  fill_seq(kv, P, sp.seq);
+  sp.batch = P.B;
+  sp.n_q = P.n_q;
+  sp.n_heads = P.H;
+  const int64_t cap = std::min<int64_t>(idx_stride, P.max_p + 1);
+  if (P.sparse_split) {
+    const int tiles = (int)((cap + kTile - 1) / kTile);
+    int n_split = std::max(1, std::min(tiles, (kManyRows + P.n_rows - 1) / P.n_rows));
+    n_split = std::min(n_split, kMaxSplit);
+    const int tiles_per = (tiles + n_split - 1) / n_split;
+    sp.split_len = tiles_per * kTile;
+    sp.n_split = (int)((cap + sp.split_len - 1) / sp.split_len);
+  } else {
+    sp.n_split = 1;
+    sp.split_len = (int)(((cap + kTile - 1) / kTile) * kTile);
+  }
+  sp.scale_log2 = scale * 1.4426950408889634f;
+  sp.q = q;
+  sp.idx = idx;
+  sp.idx_stride = idx_stride;
+  sp.count = count;
+  sp.k = kv->k;
+  sp.v = kv->v;
+  sp.k_scale = kv->k_scale;
+  sp.v_scale = kv->v_scale;
+  sp.out = out;
+  sp.out_f32 = out_f32;
+  sp.part = ws_at<float>(ws, P.off_part_sp);
+  sp.counter = ws_at<int32_t>(ws, P.off_cnt_sp);
+  sp.status = ws_at<uint32_t>(ws, P.off_status);
+  return cuda_check(launch_sparse(P.kv_dtype, sp, stream), "sparse gather attention");
+}
+
+hs2_status check_budget(int topk, int window) {
+  if (topk < 1 || topk > HS2_MAX_TOPK)
+    return fail(HS2_ERR_UNSUPPORTED, "topk %d outside [1, %d]", topk, HS2_MAX_TOPK);
+  if (window < 0 || window > HS2_MAX_WINDOW)
+    return fail(HS2_ERR_UNSUPPORTED, "window %d outside [0, %d]", window, HS2_MAX_WINDOW);
+  return HS2_OK;
+}
+
+hs2_status check_idx(const Plan &P, int topk, int window, const int32_t *idx, int idx_stride,
+                     const int32_t *count) {
+  if (!idx || !count) return fail(HS2_ERR_INVALID_ARG, "idx / count is NULL");
+  const int64_t need = std::min<int64_t>(P.max_p + 1, (int64_t)topk + window);
+  if (idx_stride < need)
+    return fail(HS2_ERR_INVALID_ARG, "idx_stride %d < %lld", idx_stride, (long long)need);
+  return HS2_OK;
+}
+
+hs2_status check_full_args(const Plan &P, const void *q, float scale, const void *out,
+                           int out_dtype, const float *lse, const float *scores,
+                           int64_t score_stride) {
+  if (!q || !out || !lse || !scores) return fail(HS2_ERR_INVALID_ARG, "q / out / lse / scores is NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(HS2_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
+  if (!valid_scale(scale)) return fail(HS2_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (out_dtype != HS2_OUT_BF16 && out_dtype != HS2_OUT_F32)
+    return fail(HS2_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  if (score_stride < P.max_p + 1)
+    return fail(HS2_ERR_INVALID_ARG, "score_stride %lld < %lld", (long long)score_stride,
+                (long long)(P.max_p + 1));
+  return HS2_OK;
+}
+
+}  // namespace
+}  // namespace hs2
+
+using namespace hs2;
+
+extern "C" {
+
+hs2_status hs2_workspace_size(const hs2_kv_view *kv, int32_t topk, int32_t window, size_t *bytes) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if ((st = check_budget(topk, window)) != HS2_OK) return st;
+  if (!bytes) return fail(HS2_ERR_INVALID_ARG, "bytes is NULL");
+  Plan P;
+  make_plan(kv, P);
+  *bytes = P.total;
+  return ok();
+}
+
+hs2_status hs2_full_attn_scores(const hs2_kv_view *kv, const void *q, float softmax_scale,
+                                void *out, int32_t out_dtype, float *lse, float *scores,
+                                int64_t score_stride, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  Plan P;
+  make_plan(kv, P);
+  if ((st = check_full_args(P, q, softmax_scale, out, out_dtype, lse, scores, score_stride)) != HS2_OK) return st;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
+  if (P.n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "multi-token query chunks (n_q > 1) are not built yet");
+  TensorMaps tm;
+  if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
+  st = run_full(kv, P, tm, q, softmax_scale, out, out_dtype == HS2_OUT_F32, lse, scores,
+                score_stride, 0, false, workspace, s);
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_topk_select(const hs2_kv_view *kv, const float *scores, int64_t score_stride,
+                           int32_t topk, int32_t window, int32_t *idx, int32_t idx_stride,
+                           int32_t *count, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if ((st = check_budget(topk, window)) != HS2_OK) return st;
+  Plan P;
+  make_plan(kv, P);
+  if (!scores) return fail(HS2_ERR_INVALID_ARG, "scores is NULL");
+  if (score_stride < P.max_p + 1)
+    return fail(HS2_ERR_INVALID_ARG, "score_stride %lld < %lld", (long long)score_stride,
+                (long long)(P.max_p + 1));
+  if ((st = check_idx(P, topk, window, idx, idx_stride, count)) != HS2_OK) return st;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
+  st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, false,
+                workspace, s);
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_sparse_gather_attn(const hs2_kv_view *kv, const void *q, const int32_t *idx,
+                                  int32_t idx_stride, const int32_t *count,
+                                  float softmax_scale, void *out, int32_t out_dtype,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  Plan P;
+  make_plan(kv, P);
+  if (!q || !out) return fail(HS2_ERR_INVALID_ARG, "q / out is NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(HS2_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
+  if (!idx || !count) return fail(HS2_ERR_INVALID_ARG, "idx / count is NULL");
+  if (idx_stride < 1) return fail(HS2_ERR_INVALID_ARG, "idx_stride %d < 1", idx_stride);
+  if (!valid_scale(softmax_scale)) return fail(HS2_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (out_dtype != HS2_OUT_BF16 && out_dtype != HS2_OUT_F32)
+    return fail(HS2_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
+  st = run_sparse(kv, P, q, idx, idx_stride, count, softmax_scale, out,
+                  out_dtype == HS2_OUT_F32, workspace, s);
+  return st == HS2_OK ? ok() : st;
+}
+
+static hs2_status block_impl(const hs2_kv_view *kv, const void *q_full,
+                             const void *const *q_sparse, int32_t n_sparse, int32_t topk,
+                             int32_t window, float softmax_scale, void *out_full,
+                             void *const *out_sparse, int32_t out_dtype, float *lse,
+                             float *scores, int64_t score_stride, int32_t *idx,
+                             int32_t idx_stride, int32_t *count, void *workspace,
+                             size_t workspace_bytes, void *const *events, int32_t n_events,
+                             void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if ((st = check_budget(topk, window)) != HS2_OK) return st;
+  Plan P;
+  make_plan(kv, P);
+  if ((st = check_full_args(P, q_full, softmax_scale, out_full, out_dtype, lse, scores, score_stride)) != HS2_OK)
+    return st;
+  if ((st = check_idx(P, topk, window, idx, idx_stride, count)) != HS2_OK) return st;
+  if (n_sparse < 0 || n_sparse > 64) return fail(HS2_ERR_INVALID_ARG, "n_sparse %d outside [0, 64]", n_sparse);
+  if (n_sparse > 0 && (!q_sparse || !out_sparse))
+    return fail(HS2_ERR_INVALID_ARG, "q_sparse / out_sparse is NULL");
+  for (int l = 0; l < n_sparse; ++l) {
+    if (!q_sparse[l] || !out_sparse[l]) return fail(HS2_ERR_INVALID_ARG, "sparse layer %d: NULL pointer", l);
+    if (!aligned16(q_sparse[l]) || !aligned16(out_sparse[l]))
+      return fail(HS2_ERR_INVALID_ARG, "sparse layer %d: q / out must be 16-byte aligned", l);
+  }
+  if (events) {
+    if (n_events != 5 + n_sparse)
+      return fail(HS2_ERR_INVALID_ARG, "n_events %d != 5 + n_sparse", n_events);
+    for (int e = 0; e < n_events; ++e)
+      if (!events[e]) return fail(HS2_ERR_INVALID_ARG, "event %d is NULL", e);
+  }
+  if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
+  if (P.n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "multi-token query chunks (n_q > 1) are not built yet");
+  TensorMaps tm;
+  if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int ev = 0;
+  const std::function<hs2_status()> mark = [&]() -> hs2_status {
+    if (!events) return HS2_OK;
+    return cuda_check(cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), s), "event record");
+  };
+  if ((st = mark()) != HS2_OK) return st;
+  if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
+  if ((st = mark()) != HS2_OK) return st;
+  const bool hist = P.n_seg > 1;
+  st = run_full(kv, P, tm, q_full, softmax_scale, out_full, out_dtype == HS2_OUT_F32, lse, scores,
+                score_stride, window, hist, workspace, s, events ? &mark : nullptr);
+  if (st != HS2_OK) return st;
+  st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, hist, workspace, s);
+  if (st != HS2_OK) return st;
+  if ((st = mark()) != HS2_OK) return st;
+  for (int l = 0; l < n_sparse; ++l) {
+    st = run_sparse(kv, P, q_sparse[l], idx, idx_stride, count, softmax_scale, out_sparse[l],
+                    out_dtype == HS2_OUT_F32, workspace, s);
+    if (st != HS2_OK) return st;
+    if ((st = mark()) != HS2_OK) return st;
+  }
+  return ok();
+}
+
+hs2_status hs2_block_decode(const hs2_kv_view *kv, const void *q_full,
+                            const void *const *q_sparse, int32_t n_sparse, int32_t topk,
+                            int32_t window, float softmax_scale, void *out_full,
+                            void *const *out_sparse, int32_t out_dtype, float *lse,
+                            float *scores, int64_t score_stride, int32_t *idx,
+                            int32_t idx_stride, int32_t *count, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+  return block_impl(kv, q_full, q_sparse, n_sparse, topk, window, softmax_scale, out_full,
+                    out_sparse, out_dtype, lse, scores, score_stride, idx, idx_stride, count,
+                    workspace, workspace_bytes, nullptr, 0, stream);
+}
+
+hs2_status hs2_block_decode_traced(const hs2_kv_view *kv, const void *q_full,
+                                   const void *const *q_sparse, int32_t n_sparse, int32_t topk,
+                                   int32_t window, float softmax_scale, void *out_full,
+                                   void *const *out_sparse, int32_t out_dtype, float *lse,
+                                   float *scores, int64_t score_stride, int32_t *idx,
+                                   int32_t idx_stride, int32_t *count, void *workspace,
+                                   size_t workspace_bytes, void *const *events,
+                                   int32_t n_events, void *stream) {
+  if (!events) return fail(HS2_ERR_INVALID_ARG, "events is NULL");
+  return block_impl(kv, q_full, q_sparse, n_sparse, topk, window, softmax_scale, out_full,
+                    out_sparse, out_dtype, lse, scores, score_stride, idx, idx_stride, count,
+                    workspace, workspace_bytes, events, n_events, stream);
+}
+
+hs2_status hs2_read_device_status(const void *workspace, void *stream) {
+  if (!workspace) return fail(HS2_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  hs2_status st = cuda_check(cudaStreamSynchronize(s), "stream synchronize");
+  if (st != HS2_OK) return st;
+  st = cuda_check(cudaMemcpy(&v, workspace, 4, cudaMemcpyDeviceToHost), "status read");
+  if (st != HS2_OK) return st;
+  if (v & kStatusTimeout) return fail(HS2_ERR_TIMEOUT, "a kernel's bounded wait ran out");
+  if (v & kStatusCheck) return fail(HS2_ERR_DEVICE_CHECK, "a kernel found an out-of-range index or count");
+  return ok();
+}
+
+const char *hs2_last_error(void) { return g_err; }
+
+const char *hs2_status_string(hs2_status s) {
+  switch (s) {
+    case HS2_OK: return "HS2_OK";
+    case HS2_ERR_INVALID_ARG: return "HS2_ERR_INVALID_ARG";
+    case HS2_ERR_UNSUPPORTED: return "HS2_ERR_UNSUPPORTED";
+    case HS2_ERR_WORKSPACE: return "HS2_ERR_WORKSPACE";
+    case HS2_ERR_CUDA: return "HS2_ERR_CUDA";
+    case HS2_ERR_DEVICE_CHECK: return "HS2_ERR_DEVICE_CHECK";
+    case HS2_ERR_TIMEOUT: return "HS2_ERR_TIMEOUT";
+  }
+  return "HS2_ERR_UNKNOWN";
+}
+
+int32_t hs2_version(void) { return HS2_VERSION; }
+
+}  // extern "C"

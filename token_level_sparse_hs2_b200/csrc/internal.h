@@ -1,0 +1,123 @@
+// internal.h -- launch parameters shared by the C-ABI layer (hs2_api.cu) and the kernels.
+// Everything a kernel needs travels by value in its parameter block (no device-side tables),
+// so every launch is self-contained and capturable.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hs2.h"
+
+namespace hs2 {
+
+constexpr int kHeadDim = 128;
+constexpr int kTile = 64;             // cache rows per pipeline tile
+constexpr int kHistBins = 2048;       // top radix digit: bits [31:21] of the fp32 score
+// device status bits (written into the workspace, read by hs2_read_device_status)
+constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusCheck = 2u;
+
+// Per-sequence geometry. Work items of sequence b are [item_begin[b], item_begin[b+1]).
+struct SeqTable {
+  int64_t start[HS2_MAX_BATCH];
+  int32_t len[HS2_MAX_BATCH];
+  int32_t item_begin[HS2_MAX_BATCH + 1];
+};
+
+// Decode (n_q == 1): full-attention pass 1 (PASS 0) and score pass 2 (PASS 1).
+struct DecodeParams {
+  SeqTable seq;
+  int32_t batch, n_heads;
+  int32_t chunk_tiles;      // 64-row tiles per work item
+  int32_t n_items;
+  int32_t window;           // pass 2: positions < p - window + 1 are top-k candidates
+  float scale_log2;         // softmax_scale * log2(e)
+  int64_t kv_rows;
+  const float *k_scale;     // FP8 per-token scales (null for bf16)
+  const float *v_scale;
+  const void *q;            // bf16 [B, H, 128]
+  void *out;                // [B, H, 128], bf16 or fp32 (pass 1)
+  int32_t out_f32;
+  float *lse;               // [B, H] (written by pass 1, read by pass 2)
+  float *scores;            // pass 2: row b at scores + b * score_stride
+  int64_t score_stride;
+  uint32_t *hist;           // pass 2: [B, kHistBins] counts of candidate top digits, or null
+  float *part;              // pass 1: [n_items, H, 2 + 128] split partials
+  int32_t *counter;         // pass 1: [B] arrival counters (self-resetting)
+  uint32_t *status;
+};
+
+// Chunk / prefill (n_q > 1): rows are (query, head) pairs, 128 per CTA (128 / H queries).
+struct RowsParams {
+  SeqTable seq;             // item_begin: row-blocks of sequence b start at rb_begin = this
+  int32_t batch, n_q, n_heads;
+  int32_t q_per_block;      // queries per row-block (128 / H)
+  int32_t n_chunks;         // kv chunks per row-block (1 = no split)
+  int32_t n_items;          // total row-blocks * n_chunks
+  float scale_log2;
+  const void *q;            // bf16 [B, n_q, H, 128]
+  void *out;                // [B, n_q, H, 128]
+  int32_t out_f32;
+  float *lse;               // [B, n_q, H]
+  float *scores;
+  int64_t score_stride;
+  float *part;              // [n_rowblocks * n_chunks, 128 rows, 2 + 128] if n_chunks > 1
+  int32_t *counter;         // [n_rowblocks]
+  uint32_t *status;
+};
+
+// Sparse gather attention: one CTA per (query row, split of the selected list).
+struct SparseParams {
+  SeqTable seq;
+  int32_t batch, n_q, n_heads;
+  int32_t n_split;          // CTAs per query row
+  int32_t split_len;        // selected entries per CTA (multiple of 64)
+  float scale_log2;
+  const void *q;            // bf16 [B, n_q, H, 128]
+  const int32_t *idx;       // [B*n_q, idx_stride]
+  int32_t idx_stride;
+  const int32_t *count;     // [B*n_q]
+  const void *k, *v;        // cache rows
+  const float *k_scale, *v_scale;
+  void *out;
+  int32_t out_f32;
+  float *part;              // [B*n_q, n_split, H, 2 + 128]
+  int32_t *counter;         // [B*n_q]
+  uint32_t *status;
+};
+
+// Top-k + window selection: n_seg CTAs per query row, each over seg_len candidate positions.
+struct TopkParams {
+  SeqTable seq;
+  int32_t batch, n_q;
+  int32_t topk, window;
+  const float *scores;
+  int64_t score_stride;
+  const uint32_t *hist;     // [B*n_q, kHistBins] top-digit counts from the score pass, or null
+  uint32_t *hist_ws;        // [B*n_q, kHistBins] built here when hist is null and n_seg > 1
+  int32_t n_seg, seg_len;
+  uint32_t *cand_key;       // [B*n_q, cand_cap] (n_seg > 1)
+  int32_t *cand_idx;
+  int32_t cand_cap;
+  int32_t *cand_count;      // [B*n_q] (self-resetting)
+  int32_t *arrive;          // [B*n_q] (self-resetting)
+  int32_t *idx;
+  int32_t idx_stride;
+  int32_t *count;
+  uint32_t *status;
+};
+
+struct TensorMaps {
+  CUtensorMap k, v;
+};
+
+// launchers (return cudaGetLastError() of the launch)
+cudaError_t launch_decode_pass(int pass, int kv_dtype, const TensorMaps &tm,
+                               const DecodeParams &p, cudaStream_t s);
+cudaError_t launch_rows_pass(int pass, int kv_dtype, const TensorMaps &tm, const RowsParams &p,
+                             cudaStream_t s);
+cudaError_t launch_sparse(int kv_dtype, const SparseParams &p, cudaStream_t s);
+cudaError_t launch_topk(const TopkParams &p, int n_rows, cudaStream_t s);
+
+}  // namespace hs2

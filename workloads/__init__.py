@@ -222,3 +222,20 @@ def sample_rows(w: Workload, n: int, seed: int = 7, extra=()) -> np.ndarray:
             must.add(b * w.n_q + int(i))
     picks = set(int(x) for x in rng.choice(total, size=min(n, total), replace=False))
     return np.asarray(sorted(must | picks), dtype=np.int64)
+
+
+def to_device(w: Workload, device="cuda"):
+    """Moves a workload's arrays to the device as torch tensors (bf16 / uint8 / fp32)."""
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+    if w.kv_dtype == "bf16":
+        k, v = bf16(w.k), bf16(w.v)
+        ks = vs = None
+    else:
+        k = torch.from_numpy(np.ascontiguousarray(w.k)).to(device)
+        v = torch.from_numpy(np.ascontiguousarray(w.v)).to(device)
+        ks = torch.from_numpy(np.ascontiguousarray(w.k_scale)).to(device)
+        vs = torch.from_numpy(np.ascontiguousarray(w.v_scale)).to(device)
+    q_full = bf16(w.q_full)
+    q_sparse = [bf16(w.q_sparse[l]) for l in range(w.n_sparse)]
+    return dict(k=k, v=v, k_scale=ks, v_scale=vs, q_full=q_full, q_sparse=q_sparse)
