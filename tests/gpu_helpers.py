@@ -17,7 +17,9 @@ O_TOL = {"bf16": 1e-2, "fp8": 3e-2}
 
 
 def run_block(w, out_dtype=torch.float32, topk=None, window=None, ws_fill=None, n_sparse=None,
-              stream=None):
+              stream=None, rows=None):
+    """Runs the block on the GPU. With `rows`, only those flat query rows are copied back and
+    the returned arrays are indexed by position in `rows`."""
     topk = w.topk if topk is None else topk
     window = w.window if window is None else window
     L = w.n_sparse if n_sparse is None else n_sparse
@@ -42,11 +44,17 @@ def run_block(w, out_dtype=torch.float32, topk=None, window=None, ws_fill=None, 
                      count, ws, topk=topk, window=window, stream=stream)
     hs2.read_device_status(ws, stream)
     torch.cuda.synchronize()
-    return dict(o_full=out_full.float().cpu().numpy().reshape(R, H, 128),
-                lse=lse.cpu().numpy().reshape(R, H),
-                scores=scores.cpu().numpy(), idx=idx.cpu().numpy(), count=count.cpu().numpy(),
-                o_sparse=[o.float().cpu().numpy().reshape(R, H, 128) for o in out_sp],
-                cache=cache, dev=d, ws=ws)
+    if rows is None:
+        sel = slice(None)
+    else:
+        sel = torch.as_tensor(np.asarray(rows), device=dev)
+    fetch = lambda t: t.reshape(R, *t.shape[2:]) if t.dim() == 4 else t
+    return dict(o_full=fetch(out_full)[sel].float().cpu().numpy(),
+                lse=lse.reshape(R, H)[sel].cpu().numpy(),
+                scores=scores[sel].cpu().numpy(), idx=idx[sel].cpu().numpy(),
+                count=count[sel].cpu().numpy(),
+                o_sparse=[fetch(o)[sel].float().cpu().numpy() for o in out_sp],
+                cache=cache, dev=d, ws=ws, rows=None if rows is None else np.asarray(rows))
 
 
 def check_scores(w, rows, s_gpu, s_ref):
@@ -63,26 +71,31 @@ def check_block(w, gpu, rows=None, topk=None, window=None, check_sparse=True):
     """Full comparison of a GPU block run against the oracle on the listed rows."""
     topk = w.topk if topk is None else topk
     window = w.window if window is None else window
-    rows = np.arange(w.n_rows) if rows is None else np.asarray(rows)
+    if gpu.get("rows") is not None:
+        rows = gpu["rows"]
+        pos = np.arange(len(rows))
+    else:
+        rows = np.arange(w.n_rows) if rows is None else np.asarray(rows)
+        pos = rows
     o_ref, lse_ref, s_ref = oracle.full_attn(w, rows=rows)
     tol = O_TOL[w.kv_dtype]
-    err = np.abs(gpu["o_full"][rows] - o_ref).max()
+    err = np.abs(gpu["o_full"][pos] - o_ref).max()
     assert err <= tol, f"O_full max-abs {err}"
-    dl = np.abs(gpu["lse"][rows] - lse_ref)
+    dl = np.abs(gpu["lse"][pos] - lse_ref)
     assert (dl <= 1e-4 + 1e-5 * np.abs(lse_ref)).all(), f"lse max diff {dl.max()}"
-    s_gpu = gpu["scores"][rows]
+    s_gpu = gpu["scores"][pos]
     check_scores(w, rows, s_gpu, s_ref)
     # selection: bit-exact against the fp32 selector on the GPU's own scores
     idx32, cnt32 = oracle.select_rows(w, rows, s_gpu, topk, window, fp32=True)
     for j, r in enumerate(rows):
         c = int(cnt32[j])
-        assert int(gpu["count"][r]) == c, (r, gpu["count"][r], c)
-        assert np.array_equal(gpu["idx"][r, :c], idx32[j, :c]), r
+        assert int(gpu["count"][pos[j]]) == c, (r, gpu["count"][pos[j]], c)
+        assert np.array_equal(gpu["idx"][pos[j], :c], idx32[j, :c]), r
     # agreement with the fp64 selector: >= 99.9 %, differences only at near-ties
     idx64, cnt64 = oracle.select_rows(w, rows, s_ref, topk, window)
     inter = tot = 0
     for j, r in enumerate(rows):
-        a = set(gpu["idx"][r, :gpu["count"][r]].tolist())
+        a = set(gpu["idx"][pos[j], :gpu["count"][pos[j]]].tolist())
         b = set(idx64[j, :cnt64[j]].tolist())
         inter += len(a & b)
         tot += len(b)
@@ -95,9 +108,9 @@ def check_block(w, gpu, rows=None, topk=None, window=None, check_sparse=True):
                 assert abs(s_ref[j, t] - kth) <= 1e-3 * kth, (r, t, s_ref[j, t], kth)
     assert inter >= 0.999 * tot, (inter, tot)
     if check_sparse:
-        cnt = gpu["count"][rows]
+        cnt = gpu["count"][pos]
         for l in range(len(gpu["o_sparse"])):
-            ref = oracle.sparse_attn(w, w.q_sparse[l], rows, gpu["idx"][rows], cnt)
-            err = np.abs(gpu["o_sparse"][l][rows] - ref).max()
+            ref = oracle.sparse_attn(w, w.q_sparse[l], rows, gpu["idx"][pos], cnt)
+            err = np.abs(gpu["o_sparse"][l][pos] - ref).max()
             assert err <= tol, f"sparse layer {l} max-abs {err}"
     return dict(o_ref=o_ref, lse_ref=lse_ref, s_ref=s_ref)

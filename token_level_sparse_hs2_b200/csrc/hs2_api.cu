@@ -41,6 +41,8 @@ constexpr int kSegLen = 16384;            // top-k candidates per CTA when rows 
 constexpr int kManyRows = 148;            // rows at least this many: one CTA per row
 constexpr int kCandCapGlobal = 8192;
 constexpr int kMaxSplit = 32;             // sparse-layer CTAs per query row, at most
+constexpr int kRowsPerBlock = 128;        // (query, head) rows per pass-1 CTA for chunks
+constexpr int kQueriesPass2 = 8;          // queries per pass-2 CTA for chunks
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -54,14 +56,17 @@ struct Plan {
   // decode passes
   int chunk_tiles = 1, n_items = 0;
   int32_t item_begin[HS2_MAX_BATCH + 1] = {};
+  // multi-token chunks: pass-1 blocks of 128 / H queries, pass-2 blocks of 8 queries
+  int32_t blk1_begin[HS2_MAX_BATCH + 1] = {}, blk2_begin[HS2_MAX_BATCH + 1] = {};
+  int n_blk1 = 0, n_chunks1 = 1, n_blk2 = 0, n_chunks2 = 1;
   // top-k
   int n_seg = 1, seg_len = 0;
   // sparse layers: n_split chosen per call from the index capacity
   bool sparse_split = false;
   // workspace (byte offsets); [0, zero_end) is cleared at the start of every call
-  size_t off_status = 0, off_cnt_p1 = 0, off_hist = 0, off_cand_count = 0, off_arrive = 0,
+  size_t off_status = 0, off_cnt_p1 = 0, off_cnt_rows = 0, off_hist = 0, off_cand_count = 0, off_arrive = 0,
          off_cnt_sp = 0, zero_end = 0;
-  size_t off_part_p1 = 0, off_cand_key = 0, off_cand_idx = 0, off_part_sp = 0, total = 0;
+  size_t off_part_p1 = 0, off_part_rows = 0, off_cand_key = 0, off_cand_idx = 0, off_part_sp = 0, total = 0;
 };
 
 hs2_status validate_view(const hs2_kv_view *kv) {
@@ -124,6 +129,21 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
     P.n_items += (int)((tiles + P.chunk_tiles - 1) / P.chunk_tiles);
   }
   P.item_begin[P.B] = P.n_items;
+  // multi-token chunks
+  if (P.n_q > 1) {
+    const int qpb1 = kRowsPerBlock / P.H, qpb2 = kQueriesPass2;
+    P.n_blk1 = P.n_blk2 = 0;
+    for (int b = 0; b < P.B; ++b) {
+      P.blk1_begin[b] = P.n_blk1;
+      P.blk2_begin[b] = P.n_blk2;
+      P.n_blk1 += (P.n_q + qpb1 - 1) / qpb1;
+      P.n_blk2 += (P.n_q + qpb2 - 1) / qpb2;
+    }
+    P.blk1_begin[P.B] = P.n_blk1;
+    P.blk2_begin[P.B] = P.n_blk2;
+    P.n_chunks1 = std::max(1, std::min(64, (kTargetItems + P.n_blk1 - 1) / P.n_blk1));
+    P.n_chunks2 = std::max(1, std::min(64, (kTargetItems + P.n_blk2 - 1) / P.n_blk2));
+  }
   // top-k segments: split long rows when there are few of them
   const int64_t max_cand = P.max_p + 1;
   if (P.n_rows >= kManyRows) {
@@ -138,6 +158,7 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   size_t o = 0;
   P.off_status = o; o = align_up(o + 4);
   P.off_cnt_p1 = o; o = align_up(o + 4 * (size_t)P.B);
+  P.off_cnt_rows = o; o = align_up(o + 4 * (size_t)P.n_blk1);
   P.off_hist = o; o = align_up(o + (P.n_seg > 1 ? 4 * (size_t)kHistBins * P.n_rows : 0));
   P.off_cand_count = o; o = align_up(o + 4 * (size_t)P.n_rows);
   P.off_arrive = o; o = align_up(o + 4 * (size_t)P.n_rows);
@@ -145,6 +166,8 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   P.zero_end = o;
   const size_t part_row = (size_t)P.H * (2 + kHeadDim) * 4;
   P.off_part_p1 = o; o = align_up(o + (P.n_q == 1 ? part_row * P.n_items : 0));
+  P.off_part_rows = o;
+  o = align_up(o + (P.n_chunks1 > 1 ? (size_t)P.n_blk1 * P.n_chunks1 * kRowsPerBlock * (2 + kHeadDim) * 4 : 0));
   const size_t cand = (P.n_seg > 1) ? (size_t)P.n_rows * kCandCapGlobal * 4 : 0;
   P.off_cand_key = o; o = align_up(o + cand);
   P.off_cand_idx = o; o = align_up(o + cand);
@@ -239,8 +262,48 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
                     float scale, void *out, int out_f32, float *lse, float *scores,
                     int64_t score_stride, int window, bool with_hist, void *ws,
                     cudaStream_t stream, const std::function<hs2_status()> *mark = nullptr) {
-  if (P.n_q != 1)
-    return fail(HS2_ERR_UNSUPPORTED, "multi-token query chunks (n_q > 1) are not built yet");
+  if (P.n_q != 1) {
+    RowsParams rp;
+    memset(&rp, 0, sizeof rp);
+    rp.batch = P.B;
+    rp.n_q = P.n_q;
+    rp.n_heads = P.H;
+    rp.scale_log2 = scale * 1.4426950408889634f;
+    rp.kv_rows = kv->kv_rows;
+    rp.k_scale = kv->k_scale;
+    rp.v_scale = kv->v_scale;
+    rp.q = q;
+    rp.out = out;
+    rp.out_f32 = out_f32;
+    rp.lse = lse;
+    rp.scores = scores;
+    rp.score_stride = score_stride;
+    rp.part = ws_at<float>(ws, P.off_part_rows);
+    rp.counter = ws_at<int32_t>(ws, P.off_cnt_rows);
+    rp.status = ws_at<uint32_t>(ws, P.off_status);
+    for (int b = 0; b < P.B; ++b) {
+      rp.seq.start[b] = kv->kv_start[b];
+      rp.seq.len[b] = kv->kv_len[b];
+    }
+    RowsParams r1 = rp, r2 = rp;
+    for (int b = 0; b <= P.B; ++b) {
+      r1.seq.item_begin[b] = P.blk1_begin[b];
+      r2.seq.item_begin[b] = P.blk2_begin[b];
+    }
+    r1.q_per_block = kRowsPerBlock / P.H;
+    r1.n_chunks = P.n_chunks1;
+    r1.n_items = P.n_blk1 * P.n_chunks1;
+    r2.q_per_block = kQueriesPass2;
+    r2.n_chunks = P.n_chunks2;
+    r2.n_items = P.n_blk2 * P.n_chunks2;
+    hs2_status st = cuda_check(launch_rows_pass(0, P.kv_dtype, tm, r1, stream), "chunk pass 1");
+    if (st != HS2_OK) return st;
+    if (mark && (st = (*mark)()) != HS2_OK) return st;
+    st = cuda_check(launch_rows_pass(1, P.kv_dtype, tm, r2, stream), "chunk score pass 2");
+    if (st != HS2_OK) return st;
+    if (mark && (st = (*mark)()) != HS2_OK) return st;
+    return HS2_OK;
+  }
   DecodeParams dp;
   memset(&dp, 0, sizeof dp);
   fill_seq(kv, P, dp.seq);
@@ -399,7 +462,6 @@ hs2_status hs2_full_attn_scores(const hs2_kv_view *kv, const void *q, float soft
   make_plan(kv, P);
   if ((st = check_full_args(P, q, softmax_scale, out, out_dtype, lse, scores, score_stride)) != HS2_OK) return st;
   if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
-  if (P.n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "multi-token query chunks (n_q > 1) are not built yet");
   TensorMaps tm;
   if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -485,7 +547,6 @@ static hs2_status block_impl(const hs2_kv_view *kv, const void *q_full,
       if (!events[e]) return fail(HS2_ERR_INVALID_ARG, "event %d is NULL", e);
   }
   if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
-  if (P.n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "multi-token query chunks (n_q > 1) are not built yet");
   TensorMaps tm;
   if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

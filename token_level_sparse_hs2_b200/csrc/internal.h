@@ -48,22 +48,26 @@ struct DecodeParams {
   uint32_t *status;
 };
 
-// Chunk / prefill (n_q > 1): rows are (query, head) pairs, 128 per CTA (128 / H queries).
+// Chunk / prefill (n_q > 1). Pass 1: blocks of 128 (query, head) rows (128 / H queries);
+// pass 2: blocks of 8 queries. Each block's causal prefix is cut into n_chunks work items.
 struct RowsParams {
-  SeqTable seq;             // item_begin: row-blocks of sequence b start at rb_begin = this
+  SeqTable seq;             // item_begin[b]: first block of sequence b
   int32_t batch, n_q, n_heads;
-  int32_t q_per_block;      // queries per row-block (128 / H)
-  int32_t n_chunks;         // kv chunks per row-block (1 = no split)
-  int32_t n_items;          // total row-blocks * n_chunks
+  int32_t q_per_block;      // queries per block
+  int32_t n_chunks;         // kv chunks per block (1 = no split)
+  int32_t n_items;          // blocks * n_chunks
   float scale_log2;
+  int64_t kv_rows;
+  const float *k_scale;     // FP8 per-token scales (null for bf16)
+  const float *v_scale;
   const void *q;            // bf16 [B, n_q, H, 128]
   void *out;                // [B, n_q, H, 128]
   int32_t out_f32;
   float *lse;               // [B, n_q, H]
-  float *scores;
+  float *scores;            // row (b * n_q + i) at scores + row * score_stride
   int64_t score_stride;
-  float *part;              // [n_rowblocks * n_chunks, 128 rows, 2 + 128] if n_chunks > 1
-  int32_t *counter;         // [n_rowblocks]
+  float *part;              // pass 1, n_chunks > 1: [blocks, n_chunks, 128, 2 + 128]
+  int32_t *counter;         // pass 1: [blocks] arrival counters (self-resetting)
   uint32_t *status;
 };
 
