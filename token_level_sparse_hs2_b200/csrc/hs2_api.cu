@@ -335,9 +335,26 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   return HS2_OK;
 }
 
+// Device scratch the selection step uses (pointers into a workspace).
+struct TopkScratch {
+  uint32_t *status = nullptr, *hist = nullptr, *cand_key = nullptr;
+  int32_t *cand_idx = nullptr, *cand_count = nullptr, *arrive = nullptr;
+};
+
+TopkScratch topk_scratch(const Plan &P, void *ws) {
+  TopkScratch t;
+  t.status = ws_at<uint32_t>(ws, P.off_status);
+  t.hist = ws_at<uint32_t>(ws, P.off_hist);
+  t.cand_key = ws_at<uint32_t>(ws, P.off_cand_key);
+  t.cand_idx = ws_at<int32_t>(ws, P.off_cand_idx);
+  t.cand_count = ws_at<int32_t>(ws, P.off_cand_count);
+  t.arrive = ws_at<int32_t>(ws, P.off_arrive);
+  return t;
+}
+
 hs2_status run_topk(const hs2_kv_view *kv, const Plan &P, const float *scores,
                     int64_t score_stride, int topk, int window, int32_t *idx, int idx_stride,
-                    int32_t *count, bool hist_ready, void *ws, cudaStream_t stream) {
+                    int32_t *count, bool hist_ready, const TopkScratch &sc, cudaStream_t stream) {
   TopkParams tp;
   memset(&tp, 0, sizeof tp);
   fill_seq(kv, P, tp.seq);
@@ -350,18 +367,18 @@ hs2_status run_topk(const hs2_kv_view *kv, const Plan &P, const float *scores,
   tp.n_seg = P.n_seg;
   tp.seg_len = P.seg_len;
   if (P.n_seg > 1) {
-    if (hist_ready) tp.hist = ws_at<uint32_t>(ws, P.off_hist);
-    else tp.hist_ws = ws_at<uint32_t>(ws, P.off_hist);
+    if (hist_ready) tp.hist = sc.hist;
+    else tp.hist_ws = sc.hist;
   }
-  tp.cand_key = ws_at<uint32_t>(ws, P.off_cand_key);
-  tp.cand_idx = ws_at<int32_t>(ws, P.off_cand_idx);
+  tp.cand_key = sc.cand_key;
+  tp.cand_idx = sc.cand_idx;
   tp.cand_cap = kCandCapGlobal;
-  tp.cand_count = ws_at<int32_t>(ws, P.off_cand_count);
-  tp.arrive = ws_at<int32_t>(ws, P.off_arrive);
+  tp.cand_count = sc.cand_count;
+  tp.arrive = sc.arrive;
   tp.idx = idx;
   tp.idx_stride = idx_stride;
   tp.count = count;
-  tp.status = ws_at<uint32_t>(ws, P.off_status);
+  tp.status = sc.status;
   return cuda_check(launch_topk(tp, P.n_rows, stream), "top-k selection");
 }
 
@@ -489,7 +506,7 @@ hs2_status hs2_topk_select(const hs2_kv_view *kv, const float *scores, int64_t s
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
   st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, false,
-                workspace, s);
+                topk_scratch(P, workspace), s);
   return st == HS2_OK ? ok() : st;
 }
 
@@ -562,7 +579,8 @@ static hs2_status block_impl(const hs2_kv_view *kv, const void *q_full,
   st = run_full(kv, P, tm, q_full, softmax_scale, out_full, out_dtype == HS2_OUT_F32, lse, scores,
                 score_stride, window, hist, workspace, s, events ? &mark : nullptr);
   if (st != HS2_OK) return st;
-  st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, hist, workspace, s);
+  st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, hist,
+                topk_scratch(P, workspace), s);
   if (st != HS2_OK) return st;
   if ((st = mark()) != HS2_OK) return st;
   for (int l = 0; l < n_sparse; ++l) {
