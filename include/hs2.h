@@ -48,6 +48,7 @@ extern "C" {
 #define HS2_MAX_BATCH 128     /* sequences per call */
 #define HS2_MAX_TOPK 2048     /* global selection budget per query row */
 #define HS2_MAX_WINDOW 4096   /* forced recent window per query row */
+#define HS2_NOALLOC_SCRATCH_BYTES (4u << 20)  /* built-in scratch of hs2_topk_select_noalloc */
 
 typedef enum {
   HS2_OK = 0,
@@ -155,6 +156,29 @@ hs2_status hs2_block_decode_traced(const hs2_kv_view *kv, const void *q_full,
                                    int32_t idx_stride, int32_t *count, void *workspace,
                                    size_t workspace_bytes, void *const *events,
                                    int32_t n_events, void *stream);
+
+/* hs2_topk_select without a caller workspace. The pages have no counterpart to this call: it
+ * is plumbing for callers that cannot allocate device memory -- for example a plugin hosted by
+ * a runtime that has already reserved the whole device for its own memory pool, or a
+ * latency-critical path that must not call cudaMalloc (which may synchronise the device).
+ * Instead of a workspace it uses a scratch array of HS2_NOALLOC_SCRATCH_BYTES (4 MiB) that the
+ * library declares as a static device variable: every GPU that loads libhs2 holds those 4 MiB
+ * until the process exits. It calls no allocator (no cudaMalloc / cudaFree). Arguments, layouts
+ * and results are those of hs2_topk_select.
+ *  - The first call on each device looks up the scratch array's device address (with that
+ *    device current) and caches it; make that first call before any stream capture.
+ *  - Calls whose selection needs more scratch than the array holds (many long rows split over
+ *    several CTAs) return HS2_ERR_WORKSPACE with the required size; use hs2_topk_select then.
+ *  - All calls share the one array and it keeps the last call's contents (the parts that must
+ *    start at zero are cleared on the stream at the start of each call). Calls that can
+ *    overlap on the GPU -- on different streams, or from different host threads -- race on it
+ *    and must be serialised by the caller.
+ *  - Errors the kernels detect themselves are recorded in the shared array and are not
+ *    reported by hs2_read_device_status. */
+hs2_status hs2_topk_select_noalloc(const hs2_kv_view *kv, const float *scores,
+                                   int64_t score_stride, int32_t topk, int32_t window,
+                                   int32_t *idx, int32_t idx_stride, int32_t *count,
+                                   void *stream);
 
 /* Synchronises `stream` and returns the status the kernels of the last call on this workspace
  * recorded: HS2_OK, HS2_ERR_TIMEOUT or HS2_ERR_DEVICE_CHECK (HS2_ERR_CUDA if the read fails). */

@@ -156,3 +156,15 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(mod, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         mod.lib()
+
+
+def test_noalloc_selection_rejects_oversized_calls(L):
+    # 100 rows of 20,000 tokens are split over several CTAs each and need far more than the
+    # built-in 4 MiB of scratch: rejected on the host with the size
+    c = cpu_cache(batch=100, lens=tuple([20000] * 100))
+    scores = torch.zeros((100, 20000))
+    idx = torch.zeros((100, 1152), dtype=torch.int32)
+    cnt = torch.zeros(100, dtype=torch.int32)
+    st = hs2.lib().hs2_topk_select_noalloc(c.ref(), scores.data_ptr(), 20000, 1024, 128,
+                                           idx.data_ptr(), 1152, cnt.data_ptr(), None)
+    assert st == 3 and b"scratch" in hs2.lib().hs2_last_error()

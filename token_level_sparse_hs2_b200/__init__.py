@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
                                        P, P, SZ, P]
         L.hs2_block_decode_traced.argtypes = [V, P, P, I32, I32, I32, F, P, P, I32, P, P, I64, P,
                                               I32, P, P, SZ, P, I32, P]
+        L.hs2_topk_select_noalloc.argtypes = [V, P, I64, I32, I32, P, I32, P, P]
         L.hs2_read_device_status.argtypes = [P, P]
         L.hs2_last_error.restype = ctypes.c_char_p
         L.hs2_status_string.restype = ctypes.c_char_p
@@ -85,7 +86,7 @@ def lib() -> ctypes.CDLL:
         L.hs2_version.restype = I32
         for name in ("hs2_workspace_size", "hs2_full_attn_scores", "hs2_topk_select",
                      "hs2_sparse_gather_attn", "hs2_block_decode", "hs2_block_decode_traced",
-                     "hs2_read_device_status"):
+                     "hs2_topk_select_noalloc", "hs2_read_device_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -175,6 +176,15 @@ def topk_select(cache: KvCache, scores, idx, count, workspace, topk=TOPK, window
     _check(lib().hs2_topk_select(cache.ref(), _ptr(scores), scores.stride(0), topk, window,
                                  _ptr(idx), idx.stride(0), _ptr(count), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def topk_select_noalloc(cache: KvCache, scores, idx, count, topk=TOPK, window=WINDOW,
+                        stream=None):
+    """topk_select for callers that cannot allocate: uses the library's built-in 4 MiB device
+    scratch instead of a workspace (see hs2_topk_select_noalloc in include/hs2.h)."""
+    _check(lib().hs2_topk_select_noalloc(cache.ref(), _ptr(scores), scores.stride(0), topk,
+                                         window, _ptr(idx), idx.stride(0), _ptr(count),
+                                         _stream(stream)))
 
 
 def sparse_gather_attn(cache: KvCache, q, idx, count, out, workspace, scale=None, stream=None):

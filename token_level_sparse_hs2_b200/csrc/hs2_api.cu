@@ -254,6 +254,56 @@ hs2_status cuda_check(cudaError_t e, const char *what) {
   return HS2_OK;
 }
 
+// ------------------------------------------------------------------ built-in selection scratch
+// Backing store of hs2_topk_select_noalloc for callers that cannot allocate. In host code the
+// name below is only a host-side stand-in for the device variable: a kernel must be given the
+// device address that cudaGetSymbolAddress returns, looked up once per device (with that
+// device current) and cached.
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[HS2_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+hs2_status noalloc_scratch(void **out) {
+  int dev = -1;
+  hs2_status st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != HS2_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return fail(HS2_ERR_UNSUPPORTED, "device %d", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    st = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+    if (st != HS2_OK) return st;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HS2_OK;
+}
+
+// Compact layout of the selection's scratch: [status, counters, histograms] are cleared per
+// call, candidate buffers are not.
+struct NoallocLayout {
+  size_t off_status, off_cand_count, off_arrive, off_hist, zero_end, off_cand_key, off_cand_idx,
+      total;
+};
+
+NoallocLayout noalloc_layout(const Plan &P) {
+  NoallocLayout L;
+  size_t o = 0;
+  L.off_status = o; o = align_up(o + 4);
+  L.off_cand_count = o; o = align_up(o + 4 * (size_t)P.n_rows);
+  L.off_arrive = o; o = align_up(o + 4 * (size_t)P.n_rows);
+  L.off_hist = o; o = align_up(o + (P.n_seg > 1 ? 4 * (size_t)kHistBins * P.n_rows : 0));
+  L.zero_end = o;
+  const size_t cand = (P.n_seg > 1) ? (size_t)P.n_rows * kCandCapGlobal * 4 : 0;
+  L.off_cand_key = o; o = align_up(o + cand);
+  L.off_cand_idx = o; o = align_up(o + cand);
+  L.total = o;
+  return L;
+}
+
 bool valid_scale(float s) { return std::isfinite(s) && s > 0.f; }
 
 // ------------------------------------------------------------------ steps
@@ -507,6 +557,40 @@ hs2_status hs2_topk_select(const hs2_kv_view *kv, const float *scores, int64_t s
   if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
   st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, false,
                 topk_scratch(P, workspace), s);
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_topk_select_noalloc(const hs2_kv_view *kv, const float *scores,
+                                   int64_t score_stride, int32_t topk, int32_t window,
+                                   int32_t *idx, int32_t idx_stride, int32_t *count,
+                                   void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if ((st = check_budget(topk, window)) != HS2_OK) return st;
+  Plan P;
+  make_plan(kv, P);
+  if (!scores) return fail(HS2_ERR_INVALID_ARG, "scores is NULL");
+  if (score_stride < P.max_p + 1)
+    return fail(HS2_ERR_INVALID_ARG, "score_stride %lld < %lld", (long long)score_stride,
+                (long long)(P.max_p + 1));
+  if ((st = check_idx(P, topk, window, idx, idx_stride, count)) != HS2_OK) return st;
+  const NoallocLayout lay = noalloc_layout(P);
+  if (lay.total > HS2_NOALLOC_SCRATCH_BYTES)
+    return fail(HS2_ERR_WORKSPACE,
+                "this selection needs %zu bytes of scratch; the built-in array holds %u "
+                "(use hs2_topk_select with a workspace)", lay.total, HS2_NOALLOC_SCRATCH_BYTES);
+  void *base = nullptr;
+  if ((st = noalloc_scratch(&base)) != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_check(cudaMemsetAsync(base, 0, lay.zero_end, s), "scratch clear")) != HS2_OK) return st;
+  TopkScratch sc;
+  sc.status = ws_at<uint32_t>(base, lay.off_status);
+  sc.cand_count = ws_at<int32_t>(base, lay.off_cand_count);
+  sc.arrive = ws_at<int32_t>(base, lay.off_arrive);
+  sc.hist = ws_at<uint32_t>(base, lay.off_hist);
+  sc.cand_key = ws_at<uint32_t>(base, lay.off_cand_key);
+  sc.cand_idx = ws_at<int32_t>(base, lay.off_cand_idx);
+  st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, false, sc, s);
   return st == HS2_OK ? ok() : st;
 }
 
