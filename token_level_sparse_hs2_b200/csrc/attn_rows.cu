@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     rows_pass1_kernel(const __grid_constant__ TensorMaps tm, const __grid_constant__ RowsParams P) {
   using C = DecodeCfg<KV, 0>;
   constexpr int H = 16 * HG;
-  constexpr int PW = 2 + kHeadDim;
+  constexpr int PW = kPartRow;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   RowsSmem<KV> sm(smem_raw);
   __shared__ int s_last;
@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     *sm.abort_flag = 0;
     fence_barrier_init();
   }
+  griddep_launch_dependents();
+  griddep_wait();
   if (KV == kKvBf16) {
     for (int t = threadIdx.x; t < kBlockRows * 16; t += kRowThreads) {
       const int r = t >> 4, ch = t & 15;
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 #pragma unroll
       for (int n = 0; n < 16; ++n)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) pr[2 + o_col<KV>(n, e, c)] = st.o[n][2 * hh + e] * st.vref;
+        for (int e = 0; e < 2; ++e) pr[kPartO + o_col<KV>(n, e, c)] = st.o[n][2 * hh + e] * st.vref;
       if (c == 0) {
         pr[0] = st.m[hh];
         pr[1] = st.l[hh];
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       const float m = __ldcg(pp);
       const float f = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
       L += f * __ldcg(pp + 1);
-      O += f * __ldcg(pp + 2 + d);
+      O += f * __ldcg(pp + kPartO + d);
     }
     const size_t orow = ((size_t)G.b * P.n_q + G.i0) * H + r;
     const float val = O / L;
@@ -253,22 +255,6 @@ struct RowsSmem2 {
   static constexpr size_t bytes() { return 1024 + C::kStages * C::kStageBytes + 2 * C::kStages * 8 + 16; }
 };
 
-// bf16 A fragments straight from global memory (rows row0.. of a [*, 128] bf16 array)
-__device__ __forceinline__ void load_q_frags_bf16_global(const __nv_bfloat16 *q, int row0,
-                                                         uint32_t (&qa)[8][4]) {
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const uint32_t *r0 = reinterpret_cast<const uint32_t *>(q + (size_t)(row0 + g) * kHeadDim);
-  const uint32_t *r1 = reinterpret_cast<const uint32_t *>(q + (size_t)(row0 + g + 8) * kHeadDim);
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    qa[ks][0] = r0[ks * 8 + c];
-    qa[ks][1] = r1[ks * 8 + c];
-    qa[ks][2] = r0[ks * 8 + 4 + c];
-    qa[ks][3] = r1[ks * 8 + 4 + c];
-  }
-}
-
 template <int KV, int HG>
 __global__ void __launch_bounds__(kRowThreads, 1)
     rows_pass2_kernel(const __grid_constant__ TensorMaps tm, const __grid_constant__ RowsParams P) {
@@ -286,6 +272,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
     *sm.abort_flag = 0;
     fence_barrier_init();
   }
+  griddep_launch_dependents();
+  griddep_wait();   // lse comes from pass 1
   __syncthreads();
   if (warp == kRowWarps) {
     produce<KV, 1>(tm, P.k_scale, P.v_scale, P.kv_rows, sm.stages, sm.full, sm.empty,
@@ -382,13 +370,15 @@ cudaError_t launch_rows_t(int pass, const TensorMaps &tm, const RowsParams &p, c
     auto kern = rows_pass1_kernel<KV, HG>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<p.n_items, kRowThreads, smem, s>>>(tm, p);
+    e = launch_pdl(kern, p.n_items, kRowThreads, smem, s, tm, p);
+    if (e != cudaSuccess) return e;
   } else {
     constexpr size_t smem = RowsSmem2<KV>::bytes();
     auto kern = rows_pass2_kernel<KV, HG>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<p.n_items, kRowThreads, smem, s>>>(tm, p);
+    e = launch_pdl(kern, p.n_items, kRowThreads, smem, s, tm, p);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -88,6 +88,22 @@ __device__ __forceinline__ void load_q_frags_bf16(uint32_t q_smem, int rows, int
   }
 }
 
+// bf16 A fragments straight from global memory (rows row0.. of a [*, 128] bf16 array)
+__device__ __forceinline__ void load_q_frags_bf16_global(const __nv_bfloat16 *q, int row0,
+                                                         uint32_t (&qa)[8][4]) {
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const uint32_t *r0 = reinterpret_cast<const uint32_t *>(q + (size_t)(row0 + g) * kHeadDim);
+  const uint32_t *r1 = reinterpret_cast<const uint32_t *>(q + (size_t)(row0 + g + 8) * kHeadDim);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    qa[ks][0] = r0[ks * 8 + c];
+    qa[ks][1] = r1[ks * 8 + c];
+    qa[ks][2] = r0[ks * 8 + 4 + c];
+    qa[ks][3] = r1[ks * 8 + 4 + c];
+  }
+}
+
 // e4m3 path: f16 A fragments (dim order of the e4m3 K fragments) of head rows
 // [row0, row0+16) of a bf16 [H][128] global array, each head scaled by 2^-e_h (exact).
 // Returns the two per-row factors 2^e_h in pow_row.
@@ -210,7 +226,7 @@ __device__ __forceinline__ void pv_tile(const uint32_t (&pa)[NT / 2][4], uint32_
 struct WarpSoftmax {
   float m[2];       // running max of the log2-domain logits
   float l[2];       // this lane's part of the running denominator
-  float vref;       // e4m3 path: V scale unit of the accumulator (1 for bf16)
+  float vref;       // e4m3 path: V-scale unit of the accumulator (starts at 1; always 1 for bf16)
   float o[16][4];   // output accumulator fragments
 
   __device__ __forceinline__ void init() {
@@ -226,6 +242,13 @@ struct WarpSoftmax {
 
 // One online-softmax step. s holds raw dot products; x = s * rowf[row] * colk[col] is the
 // log2-domain logit; invalid columns are -inf. colv: per-column V scale (e4m3) or unused.
+//
+// st.m is a reference, not necessarily the running max: it only moves (and the accumulator is
+// rescaled) when some row's tile max exceeds it by more than kLazy, so P = 2^(x - m) stays
+// below 2^kLazy (bf16 P: 2^8; f16 P: 2^4). The result is unchanged: O and the denominator
+// share the reference, and the final log-sum-exp is m + log2(l). For e4m3 caches the V-scale
+// reference st.vref likewise only moves when the tile's largest scale leaves
+// [vref * 2^-8, vref * 2^11], which keeps P * v_scale / vref within f16 range.
 template <int KV, int NT>
 __device__ __forceinline__ void softmax_pv_tile(WarpSoftmax &st, float (&s)[NT][4],
                                                 const float (&rowf)[2],
@@ -233,6 +256,7 @@ __device__ __forceinline__ void softmax_pv_tile(WarpSoftmax &st, float (&s)[NT][
                                                 const float (&colv)[NT][2],
                                                 const bool (&valid)[NT][2], uint32_t v_smem,
                                                 int tok0) {
+  constexpr float kLazy = (KV == kKvBf16) ? 8.f : 4.f;
   float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
   for (int n = 0; n < NT; ++n)
@@ -243,34 +267,44 @@ __device__ __forceinline__ void softmax_pv_tile(WarpSoftmax &st, float (&s)[NT][
       s[n][e] = x;
       mx[e >> 1] = fmaxf(mx[e >> 1], x);
     }
-  float alpha[2], mref[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
     mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-    const float mnew = fmaxf(st.m[h], mx[h]);
-    mref[h] = (mnew == -INFINITY) ? 0.f : mnew;   // nothing valid yet: p = 0 below
-    alpha[h] = fast_exp2(st.m[h] - mref[h]);       // st.m = -inf gives 0
-    st.m[h] = mnew;
   }
+  const bool keep = __all_sync(0xffffffffu, mx[0] <= st.m[0] + kLazy && mx[1] <= st.m[1] + kLazy);
+  float alpha[2] = {1.f, 1.f};
+  if (!keep) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float mnew = fmaxf(st.m[h], mx[h]);
+      const float mref = (mnew == -INFINITY) ? 0.f : mnew;   // nothing valid yet: p = 0 below
+      alpha[h] = fast_exp2(st.m[h] - mref);                  // st.m = -inf gives 0
+      st.m[h] = (mnew == -INFINITY) ? -INFINITY : mref;
+    }
+  }
+  const float mref0 = (st.m[0] == -INFINITY) ? 0.f : st.m[0];
+  const float mref1 = (st.m[1] == -INFINITY) ? 0.f : st.m[1];
   float vmul[NT][2];
   float ofix = 1.f;
   if (KV == kKvFp8) {
-    // reference V scale of this tile: the largest over its columns (whole warp)
     float vmax = 0.f;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) vmax = fmaxf(vmax, fmaxf(colv[n][0], colv[n][1]));
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) vmax = fmaxf(vmax, valid[n][e] ? colv[n][e] : 0.f);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-    if (vmax <= 0.f) vmax = 1.f;
-    const float inv = 1.f / vmax;
+    if (vmax > 0.f && (vmax > st.vref * 2048.f || vmax < st.vref * (1.f / 256.f))) {
+      ofix = st.vref / vmax;   // the accumulator moves to units of vmax
+      st.vref = vmax;
+    }
+    const float inv = 1.f / st.vref;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       vmul[n][0] = colv[n][0] * inv;
       vmul[n][1] = colv[n][1] * inv;
     }
-    ofix = st.vref * inv;   // accumulator moves to units of vmax
-    st.vref = vmax;
   }
   uint32_t pa[NT / 2][4];
   float rs[2] = {0.f, 0.f};
@@ -279,7 +313,7 @@ __device__ __forceinline__ void softmax_pv_tile(WarpSoftmax &st, float (&s)[NT][
     float p[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      p[e] = fast_exp2(s[n][e] - mref[e >> 1]);
+      p[e] = fast_exp2(s[n][e] - ((e >> 1) ? mref1 : mref0));
       rs[e >> 1] += p[e];
       if (KV == kKvFp8) p[e] *= vmul[n][e & 1];
     }
@@ -294,12 +328,14 @@ __device__ __forceinline__ void softmax_pv_tile(WarpSoftmax &st, float (&s)[NT][
 #pragma unroll
   for (int h = 0; h < 2; ++h) st.l[h] = st.l[h] * alpha[h] + rs[h];
   const float a0 = alpha[0] * ofix, a1 = alpha[1] * ofix;
+  if (!__all_sync(0xffffffffu, a0 == 1.f && a1 == 1.f)) {
 #pragma unroll
-  for (int n = 0; n < 16; ++n) {
-    st.o[n][0] *= a0;
-    st.o[n][1] *= a0;
-    st.o[n][2] *= a1;
-    st.o[n][3] *= a1;
+    for (int n = 0; n < 16; ++n) {
+      st.o[n][0] *= a0;
+      st.o[n][1] *= a0;
+      st.o[n][2] *= a1;
+      st.o[n][3] *= a1;
+    }
   }
   pv_tile<KV, NT>(pa, v_smem, tok0, st.o);
 }

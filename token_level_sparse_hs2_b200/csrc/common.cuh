@@ -190,8 +190,36 @@ __device__ __forceinline__ void record_status(uint32_t *status, uint32_t bits) {
 }  // namespace hs2
 
 namespace hs2 {
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start while the previous kernel in the stream is still running; griddep_wait() blocks until
+// that kernel has completed and its writes are visible (a no-op without the attribute), and
+// griddep_launch_dependents() lets the next kernel in the stream start early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // bar.sync on a named barrier (id 1..15) among `threads` threads (multiple of 32)
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+}  // namespace hs2
+
+namespace hs2 {
+// Launches `kernel` with programmatic stream serialization allowed (see griddep_wait).
+template <class Kernel, class... Args>
+cudaError_t launch_pdl(Kernel kernel, int grid, int block, size_t smem, cudaStream_t s,
+                       const Args &...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 }  // namespace hs2

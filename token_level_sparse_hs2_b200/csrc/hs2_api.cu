@@ -36,7 +36,8 @@ hs2_status ok() {
   return HS2_OK;
 }
 
-constexpr int kTargetItems = 4 * 148;     // decode work items per pass (~4 per SM)
+constexpr int kTargetItems = 4 * 148;     // chunk work items per pass (~4 per SM)
+constexpr int kMaxStreamCtas = 296;       // persistent decode grid, at most
 constexpr int kSegLen = 16384;            // top-k candidates per CTA when rows are split
 constexpr int kManyRows = 148;            // rows at least this many: one CTA per row
 constexpr int kCandCapGlobal = 8192;
@@ -53,9 +54,9 @@ struct Plan {
   int B = 0, n_q = 0, H = 0, kv_dtype = 0;
   int64_t kv_rows = 0, max_p = 0;
   int n_rows = 0;
-  // decode passes
-  int chunk_tiles = 1, n_items = 0;
-  int32_t item_begin[HS2_MAX_BATCH + 1] = {};
+  // decode passes: concatenated 64-row tile list of all sequences
+  int total_tiles = 0;
+  int32_t tile_begin[HS2_MAX_BATCH + 1] = {};
   // multi-token chunks: pass-1 blocks of 128 / H queries, pass-2 blocks of 8 queries
   int32_t blk1_begin[HS2_MAX_BATCH + 1] = {}, blk2_begin[HS2_MAX_BATCH + 1] = {};
   int n_blk1 = 0, n_chunks1 = 1, n_blk2 = 0, n_chunks2 = 1;
@@ -64,7 +65,7 @@ struct Plan {
   // sparse layers: n_split chosen per call from the index capacity
   bool sparse_split = false;
   // workspace (byte offsets); [0, zero_end) is cleared at the start of every call
-  size_t off_status = 0, off_cnt_p1 = 0, off_cnt_rows = 0, off_hist = 0, off_cand_count = 0, off_arrive = 0,
+  size_t off_status = 0, off_cnt_rows = 0, off_hist = 0, off_cand_count = 0, off_arrive = 0,
          off_cnt_sp = 0, zero_end = 0;
   size_t off_part_p1 = 0, off_part_rows = 0, off_cand_key = 0, off_cand_idx = 0, off_part_sp = 0, total = 0;
 };
@@ -113,22 +114,14 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   P.kv_rows = kv->kv_rows;
   P.n_rows = P.B * P.n_q;
   P.max_p = 0;
-  int64_t total_tiles = 0;
+  P.total_tiles = 0;
   for (int b = 0; b < P.B; ++b) {
     P.max_p = std::max<int64_t>(P.max_p, kv->kv_len[b] - 1);
     const int64_t r0 = kv->kv_start[b], r1 = r0 + kv->kv_len[b];
-    total_tiles += (r1 + kTile - 1) / kTile - r0 / kTile;
+    P.tile_begin[b] = P.total_tiles;   // decode: tiles of every sequence, concatenated
+    P.total_tiles += (int)((r1 + kTile - 1) / kTile - r0 / kTile);
   }
-  // decode items: chunks of chunk_tiles tiles per sequence
-  P.chunk_tiles = (int)std::max<int64_t>(1, (total_tiles + kTargetItems - 1) / kTargetItems);
-  P.n_items = 0;
-  for (int b = 0; b < P.B; ++b) {
-    const int64_t r0 = kv->kv_start[b], r1 = r0 + kv->kv_len[b];
-    const int64_t tiles = (r1 + kTile - 1) / kTile - r0 / kTile;
-    P.item_begin[b] = P.n_items;
-    P.n_items += (int)((tiles + P.chunk_tiles - 1) / P.chunk_tiles);
-  }
-  P.item_begin[P.B] = P.n_items;
+  P.tile_begin[P.B] = P.total_tiles;
   // multi-token chunks
   if (P.n_q > 1) {
     const int qpb1 = kRowsPerBlock / P.H, qpb2 = kQueriesPass2;
@@ -157,21 +150,22 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   // workspace layout
   size_t o = 0;
   P.off_status = o; o = align_up(o + 4);
-  P.off_cnt_p1 = o; o = align_up(o + 4 * (size_t)P.B);
   P.off_cnt_rows = o; o = align_up(o + 4 * (size_t)P.n_blk1);
   P.off_hist = o; o = align_up(o + (P.n_seg > 1 ? 4 * (size_t)kHistBins * P.n_rows : 0));
   P.off_cand_count = o; o = align_up(o + 4 * (size_t)P.n_rows);
   P.off_arrive = o; o = align_up(o + 4 * (size_t)P.n_rows);
   P.off_cnt_sp = o; o = align_up(o + 4 * (size_t)P.n_rows);
   P.zero_end = o;
-  const size_t part_row = (size_t)P.H * (2 + kHeadDim) * 4;
-  P.off_part_p1 = o; o = align_up(o + (P.n_q == 1 ? part_row * P.n_items : 0));
+  const size_t part_row = (size_t)P.H * kPartRow * 4;
+  const size_t max_slots =
+      (size_t)decode_slots_per_cta(P.H) * ((size_t)std::min(kMaxStreamCtas, P.total_tiles) + P.B);
+  P.off_part_p1 = o; o = align_up(o + (P.n_q == 1 ? part_row * max_slots : 0));
   P.off_part_rows = o;
-  o = align_up(o + (P.n_chunks1 > 1 ? (size_t)P.n_blk1 * P.n_chunks1 * kRowsPerBlock * (2 + kHeadDim) * 4 : 0));
+  o = align_up(o + (P.n_chunks1 > 1 ? (size_t)P.n_blk1 * P.n_chunks1 * kRowsPerBlock * kPartRow * 4 : 0));
   const size_t cand = (P.n_seg > 1) ? (size_t)P.n_rows * kCandCapGlobal * 4 : 0;
   P.off_cand_key = o; o = align_up(o + cand);
   P.off_cand_idx = o; o = align_up(o + cand);
-  P.off_part_sp = o; o = align_up(o + (P.sparse_split ? part_row * kMaxSplit * P.n_rows : 0));
+  P.off_part_sp = o; o = align_up(o + (P.sparse_split ? part_row * kMaxSplit * 4 * P.n_rows : 0));
   P.total = o;
 }
 
@@ -180,9 +174,9 @@ void fill_seq(const hs2_kv_view *kv, const Plan &P, SeqTable &t) {
   for (int b = 0; b < P.B; ++b) {
     t.start[b] = kv->kv_start[b];
     t.len[b] = kv->kv_len[b];
-    t.item_begin[b] = P.item_begin[b];
+    t.tile_begin[b] = P.tile_begin[b];
   }
-  t.item_begin[P.B] = P.item_begin[P.B];
+  t.tile_begin[P.B] = P.tile_begin[P.B];
 }
 
 hs2_status check_ws(const Plan &P, void *ws, size_t bytes) {
@@ -306,6 +300,26 @@ NoallocLayout noalloc_layout(const Plan &P) {
 
 bool valid_scale(float s) { return std::isfinite(s) && s > 0.f; }
 
+// multiprocessors of the current device (cached per device)
+hs2_status sm_count(int *out) {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  hs2_status st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != HS2_OK) return st;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) {
+    *out = cache[dev];
+    return HS2_OK;
+  }
+  int n = 0;
+  st = cuda_check(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev), "SM count");
+  if (st != HS2_OK) return st;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  *out = n;
+  return HS2_OK;
+}
+
 // ------------------------------------------------------------------ steps
 
 hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, const void *q,
@@ -357,10 +371,24 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   DecodeParams dp;
   memset(&dp, 0, sizeof dp);
   fill_seq(kv, P, dp.seq);
+  int sms = 0;
+  hs2_status st = sm_count(&sms);
+  if (st != HS2_OK) return st;
+  const int G = std::max(1, std::min({sms, P.total_tiles, kMaxStreamCtas}));
+  // partial slots: 4 per (CTA, sequence) pair; CTA i owns tiles [i*T/G, (i+1)*T/G)
+  const int T = P.total_tiles;
+  auto cta_of = [&](int g) { return (int)(((int64_t)(g + 1) * G - 1) / T); };
+  int slots = 0;
+  for (int b = 0; b < P.B; ++b) {
+    dp.seq.item_begin[b] = slots;
+    slots += decode_slots_per_cta(P.H) * (cta_of(P.tile_begin[b + 1] - 1) - cta_of(P.tile_begin[b]) + 1);
+  }
+  dp.seq.item_begin[P.B] = slots;
   dp.batch = P.B;
   dp.n_heads = P.H;
-  dp.chunk_tiles = P.chunk_tiles;
-  dp.n_items = P.n_items;
+  dp.total_tiles = T;
+  dp.n_ctas = G;
+  dp.n_ctas2 = std::max(1, std::min({2 * sms, P.total_tiles, kMaxStreamCtas}));
   dp.window = window;
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.kv_rows = kv->kv_rows;
@@ -374,10 +402,22 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   dp.score_stride = score_stride;
   dp.hist = with_hist ? ws_at<uint32_t>(ws, P.off_hist) : nullptr;
   dp.part = ws_at<float>(ws, P.off_part_p1);
-  dp.counter = ws_at<int32_t>(ws, P.off_cnt_p1);
   dp.status = ws_at<uint32_t>(ws, P.off_status);
-  hs2_status st = cuda_check(launch_decode_pass(0, P.kv_dtype, tm, dp, stream), "full-attention pass 1");
+  st = cuda_check(launch_decode_pass(0, P.kv_dtype, tm, dp, stream), "full-attention pass 1");
   if (st != HS2_OK) return st;
+  {
+    MergeParams mp;
+    memset(&mp, 0, sizeof mp);
+    mp.seq = dp.seq;
+    mp.by_seq = 1;
+    mp.n_groups = P.B;
+    mp.n_heads = P.H;
+    mp.part = dp.part;
+    mp.out = out;
+    mp.out_f32 = out_f32;
+    mp.lse = lse;
+    if ((st = cuda_check(launch_merge(mp, stream), "pass 1 merge")) != HS2_OK) return st;
+  }
   if (mark && (st = (*mark)()) != HS2_OK) return st;
   st = cuda_check(launch_decode_pass(1, P.kv_dtype, tm, dp, stream), "score pass 2");
   if (st != HS2_OK) return st;
@@ -467,7 +507,19 @@ hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const
   sp.part = ws_at<float>(ws, P.off_part_sp);
   sp.counter = ws_at<int32_t>(ws, P.off_cnt_sp);
   sp.status = ws_at<uint32_t>(ws, P.off_status);
-  return cuda_check(launch_sparse(P.kv_dtype, sp, stream), "sparse gather attention");
+  hs2_status st = cuda_check(launch_sparse(P.kv_dtype, sp, stream), "sparse gather attention");
+  if (st != HS2_OK || sp.n_split == 1) return st;
+  MergeParams mp;
+  memset(&mp, 0, sizeof mp);
+  mp.by_seq = 0;
+  mp.n_groups = P.n_rows;
+  mp.n_fixed = sp.n_split * (4 / (P.H / 16));   // partial slots per row: splits x token groups
+  mp.n_heads = P.H;
+  mp.part = sp.part;
+  mp.out = out;
+  mp.out_f32 = out_f32;
+  mp.lse = nullptr;
+  return cuda_check(launch_merge(mp, stream), "sparse merge");
 }
 
 hs2_status check_budget(int topk, int window) {

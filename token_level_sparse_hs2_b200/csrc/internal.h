@@ -13,24 +13,38 @@ namespace hs2 {
 
 constexpr int kHeadDim = 128;
 constexpr int kTile = 64;             // cache rows per pipeline tile
-constexpr int kHistBins = 2048;       // top radix digit: bits [31:21] of the fp32 score
+constexpr int kHistBins = 2048;
+// A split partial row: [max (log2 units), denominator, 2 pad, unnormalised output x 128];
+// 132 floats keep the output 16-byte aligned.
+constexpr int kPartRow = 4 + 128;
+constexpr int kPartO = 4;       // top radix digit: bits [31:21] of the fp32 score
+// decode pass 1: partial slots per (CTA, sequence) -- one per token group of consumer warps
+constexpr int decode_slots_per_cta(int n_heads) { return n_heads == 16 ? 8 : 4; }
+
 // device status bits (written into the workspace, read by hs2_read_device_status)
 constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusCheck = 2u;
 
-// Per-sequence geometry. Work items of sequence b are [item_begin[b], item_begin[b+1]).
+// Per-sequence geometry. Work items (or partial slots) of sequence b are
+// [item_begin[b], item_begin[b+1]); its 64-row tiles are [tile_begin[b], tile_begin[b+1]) of
+// the concatenated tile list of all sequences.
 struct SeqTable {
   int64_t start[HS2_MAX_BATCH];
   int32_t len[HS2_MAX_BATCH];
   int32_t item_begin[HS2_MAX_BATCH + 1];
+  int32_t tile_begin[HS2_MAX_BATCH + 1];
 };
 
-// Decode (n_q == 1): full-attention pass 1 (PASS 0) and score pass 2 (PASS 1).
+// Decode (n_q == 1): full-attention pass 1 (PASS 0) and score pass 2 (PASS 1). A persistent
+// grid of n_ctas CTAs; CTA i streams tiles [i*T/n_ctas, (i+1)*T/n_ctas) of the concatenated
+// list (T = total_tiles). Pass-1 partial slots of sequence b start at seq.item_begin[b]: 4 per
+// CTA that touches b.
 struct DecodeParams {
   SeqTable seq;
   int32_t batch, n_heads;
-  int32_t chunk_tiles;      // 64-row tiles per work item
-  int32_t n_items;
+  int32_t total_tiles;
+  int32_t n_ctas;           // pass-1 grid (partial slots are laid out for it)
+  int32_t n_ctas2;          // pass-2 grid
   int32_t window;           // pass 2: positions < p - window + 1 are top-k candidates
   float scale_log2;         // softmax_scale * log2(e)
   int64_t kv_rows;
@@ -43,8 +57,7 @@ struct DecodeParams {
   float *scores;            // pass 2: row b at scores + b * score_stride
   int64_t score_stride;
   uint32_t *hist;           // pass 2: [B, kHistBins] counts of candidate top digits, or null
-  float *part;              // pass 1: [n_items, H, 2 + 128] split partials
-  int32_t *counter;         // pass 1: [B] arrival counters (self-resetting)
+  float *part;              // pass 1: [slots, H, kPartRow] partials
   uint32_t *status;
 };
 
@@ -112,6 +125,19 @@ struct TopkParams {
   uint32_t *status;
 };
 
+// Merge of split partials into outputs: one CTA per (group, head). Group g owns partial slots
+// [slot_begin(g), slot_begin(g) + n(g)): from seq.item_begin when by_seq, else g * n_fixed.
+// Groups with a single slot were written directly by their CTA and are skipped.
+struct MergeParams {
+  SeqTable seq;
+  int32_t by_seq;
+  int32_t n_groups, n_fixed, n_heads;
+  const float *part;        // [slots, H, kPartRow]
+  void *out;                // [groups, H, 128]
+  int32_t out_f32;
+  float *lse;               // [groups, H] or null
+};
+
 struct TensorMaps {
   CUtensorMap k, v;
 };
@@ -123,5 +149,6 @@ cudaError_t launch_rows_pass(int pass, int kv_dtype, const TensorMaps &tm, const
                              cudaStream_t s);
 cudaError_t launch_sparse(int kv_dtype, const SparseParams &p, cudaStream_t s);
 cudaError_t launch_topk(const TopkParams &p, int n_rows, cudaStream_t s);
+cudaError_t launch_merge(const MergeParams &p, cudaStream_t s);
 
 }  // namespace hs2

@@ -31,12 +31,13 @@ namespace {
 constexpr int kThreadsTk = 512;
 constexpr int kWarpsTk = kThreadsTk / 32;
 constexpr int kCandCap = 8192;     // candidates finished in shared memory
+constexpr int kUnroll = 8;         // independent score loads in flight per thread
 
 struct TkSmem {
   uint32_t hist[kHistBins];
   uint32_t key[kCandCap];
   int32_t idx[kCandCap];
-  int32_t sel[HS2_MAX_TOPK];
+  alignas(16) int32_t sel[HS2_MAX_TOPK];
   int32_t warp_sums[kWarpsTk];
   int32_t n_cand;
   int32_t n_sel;
@@ -45,40 +46,39 @@ struct TkSmem {
   int32_t last;
 };
 
-// One warp finds the bucket holding the `need`-th element counting from the top (desc) or
-// the bottom (asc) of a histogram; result in sm.bucket / sm.above (count strictly before it).
-__device__ void find_bucket(const uint32_t *hist, int nbins, uint32_t need, bool desc,
-                            int32_t *out_bucket, uint32_t *out_before) {
-  const int lane = threadIdx.x & 31;
-  uint32_t run = 0;
-  for (int base = 0; base < nbins; base += 32) {
-    const int k = base + lane;
-    const int bin = desc ? nbins - 1 - k : k;
-    const uint32_t v = (k < nbins) ? hist[bin] : 0u;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    const uint32_t tot = __shfl_sync(0xffffffffu, x, 31);
-    if (run + tot >= need) {
-      const unsigned ball = __ballot_sync(0xffffffffu, run + x >= need);
-      const int first = __ffs(ball) - 1;
-      const uint32_t before = __shfl_sync(0xffffffffu, x - v, first);
-      if (lane == 0) {
-        const int kk = base + first;
-        *out_bucket = desc ? nbins - 1 - kk : kk;
-        *out_before = run + before;
-      }
-      return;
-    }
-    run += tot;
-  }
-  if (lane == 0) {
+// Finds the bucket holding the `need`-th element counting from the top (desc) or the bottom
+// (asc) of a histogram, and how many elements come before it. Called by all threads
+// (nbins = 1024 or 2048): each thread owns nbins / 512 consecutive positions of the scan
+// order and one block scan finds the thread whose positions hold the target. The result is
+// in *out_bucket / *out_before for every thread on return.
+__device__ int block_excl_scan(int v, int32_t *warp_sums, int *total);
+
+__device__ void find_bucket_block(const uint32_t *hist, int nbins, uint32_t need, bool desc,
+                                  int32_t *warp_sums, int32_t *out_bucket, uint32_t *out_before) {
+  const int E = nbins / kThreadsTk;
+  const int k0 = threadIdx.x * E;
+  if (threadIdx.x == 0) {   // only reached if need exceeds the total
     *out_bucket = desc ? 0 : nbins - 1;
-    *out_before = run;
+    *out_before = 0;
   }
+  uint32_t loc = 0;
+  for (int e = 0; e < E; ++e) loc += hist[desc ? nbins - 1 - (k0 + e) : k0 + e];
+  int tot;
+  const uint32_t pre = (uint32_t)block_excl_scan((int)loc, warp_sums, &tot);
+  if (pre < need && need <= pre + loc) {
+    uint32_t run = pre;
+    for (int e = 0; e < E; ++e) {
+      const int bin = desc ? nbins - 1 - (k0 + e) : k0 + e;
+      const uint32_t v = hist[bin];
+      if (run + v >= need) {
+        *out_bucket = bin;
+        *out_before = run;
+        break;
+      }
+      run += v;
+    }
+  }
+  __syncthreads();
 }
 
 // exclusive block-wide prefix sum of one int per thread; *total gets the block sum
@@ -136,7 +136,7 @@ __device__ __forceinline__ void append(bool take, uint32_t key, int32_t t, int32
 // Exact finish on n <= kCandCap candidates in shared memory that contain every candidate with
 // top digit >= B1 (above = how many have top digit > B1). Writes the ascending selection.
 __device__ void finish_from_smem(TkSmem &sm, int n, int B1, uint32_t above, int topk,
-                                 int32_t *out) {
+                                 int max_idx, int32_t *out) {
   uint32_t prefix = (uint32_t)B1 << 21, mask = 0xffe00000u;
   uint32_t need = topk - above;
   const int shifts[2] = {10, 0};
@@ -151,8 +151,7 @@ __device__ void finish_from_smem(TkSmem &sm, int n, int B1, uint32_t above, int 
       if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> sh) & (nb - 1)], 1u);
     }
     __syncthreads();
-    if (threadIdx.x < 32) find_bucket(sm.hist, nb, need, true, &sm.bucket, &sm.above);
-    __syncthreads();
+    find_bucket_block(sm.hist, nb, need, true, sm.warp_sums, &sm.bucket, &sm.above);
     const int bk = sm.bucket;
     need -= sm.above;
     prefix |= (uint32_t)bk << sh;
@@ -176,8 +175,7 @@ __device__ void finish_from_smem(TkSmem &sm, int n, int B1, uint32_t above, int 
         if (sm.key[t] == tau && (ix & imask) == iprefix) atomicAdd(&sm.hist[(ix >> sh) & (nb - 1)], 1u);
       }
       __syncthreads();
-      if (threadIdx.x < 32) find_bucket(sm.hist, nb, ineed, false, &sm.bucket, &sm.above);
-      __syncthreads();
+      find_bucket_block(sm.hist, nb, ineed, false, sm.warp_sums, &sm.bucket, &sm.above);
       ineed -= sm.above;
       iprefix |= (uint32_t)sm.bucket << sh;
       imask |= (uint32_t)(nb - 1) << sh;
@@ -210,28 +208,43 @@ __device__ void finish_from_smem(TkSmem &sm, int n, int B1, uint32_t above, int 
     }
   }
   __syncthreads();
-  // bitonic sort of the topk selected indices (ascending), padded to a power of two
-  int N = 2;
-  while (N < topk) N <<= 1;
-  for (int t = topk + threadIdx.x; t < N; t += kThreadsTk) sm.sel[t] = 0x7fffffff;
-  __syncthreads();
-  for (int k = 2; k <= N; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int t = threadIdx.x; t < N; t += kThreadsTk) {
-        const int u = t ^ j;
-        if (u > t) {
-          const int a = sm.sel[t], c = sm.sel[u];
-          const bool up = (t & k) == 0;
-          if ((a > c) == up) {
-            sm.sel[t] = c;
-            sm.sel[u] = a;
-          }
-        }
-      }
-      __syncthreads();
+  // Ascending order without a full sort: bucket the kept indices by their top bits (at most
+  // 1024 buckets), place each bucket by an exclusive scan of the bucket counts, and rank each
+  // index inside its bucket by counting the smaller members (indices are distinct).
+  {
+    uint32_t *bcnt = sm.hist, *bbeg = sm.hist + 1024;
+    int32_t *tmp = reinterpret_cast<int32_t *>(sm.key);
+    const int nbits = 32 - __clz(max(1, max_idx));
+    const int shift = max(0, nbits - 10);
+    for (int t = threadIdx.x; t < 1024; t += kThreadsTk) bcnt[t] = 0;
+    __syncthreads();
+    for (int t = threadIdx.x; t < topk; t += kThreadsTk) atomicAdd(&bcnt[sm.sel[t] >> shift], 1u);
+    __syncthreads();
+    {
+      const int e0 = 2 * threadIdx.x;
+      const int loc = (int)(bcnt[e0] + bcnt[e0 + 1]);
+      int tot;
+      const int pre = block_excl_scan(loc, sm.warp_sums, &tot);
+      bbeg[e0] = pre;
+      bbeg[e0 + 1] = pre + bcnt[e0];
     }
+    __syncthreads();
+    for (int t = threadIdx.x; t < 1024; t += kThreadsTk) bcnt[t] = 0;   // reused as fill counters
+    __syncthreads();
+    for (int t = threadIdx.x; t < topk; t += kThreadsTk) {
+      const int x = sm.sel[t], bk = x >> shift;
+      tmp[bbeg[bk] + atomicAdd(&bcnt[bk], 1u)] = x;
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < topk; t += kThreadsTk) {
+      const int x = tmp[t], bk = x >> shift;
+      const int j0 = bbeg[bk], j1 = j0 + (int)bcnt[bk];
+      int r = j0;
+      for (int j = j0; j < j1; ++j) r += tmp[j] < x;
+      out[r] = x;
+    }
+    __syncthreads();
   }
-  for (int t = threadIdx.x; t < topk; t += kThreadsTk) out[t] = sm.sel[t];
 }
 
 // Exact fallback over the whole candidate row in global memory (any number of equal keys):
@@ -246,13 +259,20 @@ __device__ void finish_from_global(TkSmem &sm, const float *s, int64_t nc, int B
     const int sh = shifts[pass], nb = 1 << widths[pass];
     for (int t = threadIdx.x; t < nb; t += kThreadsTk) sm.hist[t] = 0;
     __syncthreads();
-    for (int64_t t = threadIdx.x; t < nc; t += kThreadsTk) {
-      const uint32_t k = load_key(s, t);
-      if ((k & mask) == prefix) atomicAdd(&sm.hist[(k >> sh) & (nb - 1)], 1u);
+    for (int64_t base = 0; base < nc; base += kThreadsTk * kUnroll) {
+      uint32_t k[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t t = base + u * kThreadsTk + threadIdx.x;
+        k[u] = t < nc ? load_key(s, t) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (base + u * kThreadsTk + threadIdx.x < nc && (k[u] & mask) == prefix)
+          atomicAdd(&sm.hist[(k[u] >> sh) & (nb - 1)], 1u);
     }
     __syncthreads();
-    if (threadIdx.x < 32) find_bucket(sm.hist, nb, need, true, &sm.bucket, &sm.above);
-    __syncthreads();
+    find_bucket_block(sm.hist, nb, need, true, sm.warp_sums, &sm.bucket, &sm.above);
     need -= sm.above;
     prefix |= (uint32_t)sm.bucket << sh;
     mask |= (uint32_t)(nb - 1) << sh;
@@ -283,6 +303,8 @@ __device__ void finish_from_global(TkSmem &sm, const float *s, int64_t nc, int B
 // produce one and the row is split over several CTAs).
 __global__ void __launch_bounds__(kThreadsTk) topk_hist_kernel(const __grid_constant__ TopkParams P) {
   __shared__ uint32_t hist[kHistBins];
+  griddep_launch_dependents();
+  griddep_wait();
   const int r = blockIdx.x / P.n_seg, sg = blockIdx.x % P.n_seg;
   const int b = r / P.n_q, i = r % P.n_q;
   const int64_t p = (int64_t)P.seq.len[b] - P.n_q + i;
@@ -292,8 +314,17 @@ __global__ void __launch_bounds__(kThreadsTk) topk_hist_kernel(const __grid_cons
   __syncthreads();
   const float *s = P.scores + (size_t)r * P.score_stride;
   const int64_t s0 = (int64_t)sg * P.seg_len, s1 = min(nc, s0 + P.seg_len);
-  for (int64_t t = s0 + threadIdx.x; t < s1; t += kThreadsTk)
-    atomicAdd(&hist[load_key(s, t) >> 21], 1u);
+  for (int64_t base = s0; base < s1; base += kThreadsTk * kUnroll) {
+    uint32_t k[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t t = base + u * kThreadsTk + threadIdx.x;
+      k[u] = t < s1 ? load_key(s, t) : 0xffffffffu;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (base + u * kThreadsTk + threadIdx.x < s1) atomicAdd(&hist[k[u] >> 21], 1u);
+  }
   __syncthreads();
   uint32_t *gh = P.hist_ws + (size_t)r * kHistBins;
   for (int t = threadIdx.x; t < kHistBins; t += kThreadsTk)
@@ -303,6 +334,8 @@ __global__ void __launch_bounds__(kThreadsTk) topk_hist_kernel(const __grid_cons
 __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_constant__ TopkParams P) {
   extern __shared__ __align__(16) uint8_t tk_raw[];
   TkSmem &sm = *reinterpret_cast<TkSmem *>(tk_raw);
+  griddep_launch_dependents();
+  griddep_wait();
   const int r = blockIdx.x / P.n_seg, sg = blockIdx.x % P.n_seg;
   const int b = r / P.n_q, i = r % P.n_q;
   const int64_t p = (int64_t)P.seq.len[b] - P.n_q + i;
@@ -324,38 +357,61 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
   } else {   // single segment: build it here
     for (int t = threadIdx.x; t < kHistBins; t += kThreadsTk) sm.hist[t] = 0;
     __syncthreads();
-    for (int64_t t = threadIdx.x; t < nc; t += kThreadsTk) atomicAdd(&sm.hist[load_key(s, t) >> 21], 1u);
+    for (int64_t base = 0; base < nc; base += kThreadsTk * kUnroll) {
+      uint32_t k[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t t = base + u * kThreadsTk + threadIdx.x;
+        k[u] = t < nc ? load_key(s, t) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (base + u * kThreadsTk + threadIdx.x < nc) atomicAdd(&sm.hist[k[u] >> 21], 1u);
+    }
   }
   if (threadIdx.x == 0) sm.n_cand = 0;
   __syncthreads();
   // 2. bucket of the topk-th largest key
-  if (threadIdx.x < 32) find_bucket(sm.hist, kHistBins, (uint32_t)P.topk, true, &sm.bucket, &sm.above);
-  __syncthreads();
+  find_bucket_block(sm.hist, kHistBins, (uint32_t)P.topk, true, sm.warp_sums, &sm.bucket, &sm.above);
   const int B1 = sm.bucket;
   const uint32_t above = sm.above;
   // 3. compact every candidate of this segment with top digit >= B1
   const int64_t s0 = (int64_t)sg * P.seg_len, s1 = min(nc, s0 + P.seg_len);
-  const int64_t span = s1 - s0;
-  const int64_t steps = (span + kThreadsTk - 1) / kThreadsTk;
   int32_t *gcount = P.cand_count + r;
   uint32_t *gkey = P.cand_key + (size_t)r * P.cand_cap;
   int32_t *gidx = P.cand_idx + (size_t)r * P.cand_cap;
-  for (int64_t it = 0; it < steps; ++it) {
-    const int64_t t = s0 + it * kThreadsTk + threadIdx.x;
-    uint32_t k = 0;
-    bool take = false;
-    if (t < s1) {
-      k = load_key(s, t);
-      take = (int)(k >> 21) >= B1;
+  for (int64_t base = s0; base < s1; base += kThreadsTk * kUnroll) {
+    uint32_t k[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t t = base + u * kThreadsTk + threadIdx.x;
+      k[u] = t < s1 ? load_key(s, t) : 0u;
     }
-    if (P.n_seg == 1) append<true>(take, k, (int32_t)t, &sm.n_cand, sm.key, sm.idx, kCandCap);
-    else append<false>(take, k, (int32_t)t, gcount, gkey, gidx, P.cand_cap);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t t = base + u * kThreadsTk + threadIdx.x;
+      const bool take = t < s1 && (int)(k[u] >> 21) >= B1;
+      append<true>(take, k[u], (int32_t)t, &sm.n_cand, sm.key, sm.idx, kCandCap);
+    }
   }
+  __syncthreads();
   int n;
   if (P.n_seg == 1) {
-    __syncthreads();
     n = sm.n_cand;
   } else {
+    // publish this segment's candidates with one global reservation (the count keeps counting
+    // past the capacity, which sends the finishing CTA to the exact fallback)
+    const int nl = sm.n_cand;
+    if (threadIdx.x == 0) sm.bucket = atomicAdd(gcount, nl);
+    __syncthreads();
+    const int base = sm.bucket;
+    const int ncopy = min(nl, kCandCap);
+    for (int t = threadIdx.x; t < ncopy; t += kThreadsTk) {
+      if (base + t < P.cand_cap) {
+        gkey[base + t] = sm.key[t];
+        gidx[base + t] = sm.idx[t];
+      }
+    }
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -380,7 +436,7 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
   }
   // 4. finish
   const bool fits = (P.n_seg == 1) ? (n <= kCandCap) : (n <= kCandCap && n <= P.cand_cap);
-  if (fits) finish_from_smem(sm, n, B1, above, P.topk, out);
+  if (fits) finish_from_smem(sm, n, B1, above, P.topk, (int)(nc - 1), out);
   else finish_from_global(sm, s, nc, B1, above, P.topk, out);
   // 5. the forced window
   for (int64_t t = nc + threadIdx.x; t <= p; t += kThreadsTk) out[P.topk + (t - nc)] = (int32_t)t;
@@ -396,11 +452,11 @@ cudaError_t launch_topk(const TopkParams &p, int n_rows, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int grid = n_rows * p.n_seg;
   if (!p.hist && p.n_seg > 1) {
-    topk_hist_kernel<<<grid, kThreadsTk, 0, s>>>(p);
-    e = cudaGetLastError();
+    e = launch_pdl(topk_hist_kernel, grid, kThreadsTk, 0, s, p);
     if (e != cudaSuccess) return e;
   }
-  topk_select_kernel<<<grid, kThreadsTk, smem, s>>>(p);
+  e = launch_pdl(topk_select_kernel, grid, kThreadsTk, smem, s, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
