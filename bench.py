@@ -330,7 +330,7 @@ def main():
             traffic = json.load(f).get(w.name, {}).get("pass1")
     except Exception:
         pass
-    kernels_per_step = 2 + 1 + L   # pass 1, pass 2, selection, sparse layers
+    kernels_per_step = 4 + L   # pass 1, its merge, pass 2, selection, one per sparse layer
     line = {
         "metric": METRIC, "value": world * R / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,

@@ -362,17 +362,22 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, 2)
           colk[n][e] = (KV == kKvFp8)
                            ? reinterpret_cast<const float *>(stg + C::kKBytes)[tok0 + n * 8 + 2 * c + e]
                            : 1.f;
-      float cs[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      float sacc[HG][2][4];
+      qk_tile_mt<KV, HG, 2>(qa, smem_u32(stg), tok0, sacc);
+      // x = s * (rowf * colk) - lse2 and the sum over heads, two columns at a time
+      float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int mt = 0; mt < HG; ++mt) {
-        float sacc[2][4];
-        qk_tile<KV, 2>(qa[mt], smem_u32(stg), tok0, sacc);
+      for (int mt = 0; mt < HG; ++mt)
 #pragma unroll
         for (int n = 0; n < 2; ++n)
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            cs[n][e & 1] += fast_exp2(sacc[n][e] * rowf[mt][e >> 1] * colk[n][e & 1] - lse2[mt][e >> 1]);
-      }
+          for (int h = 0; h < 2; ++h) {
+            const float2 a = make_float2(rowf[mt][h] * colk[n][0], rowf[mt][h] * colk[n][1]);
+            const float2 x = ffma2(make_float2(sacc[mt][n][2 * h], sacc[mt][n][2 * h + 1]), a,
+                                   make_float2(-lse2[mt][h], -lse2[mt][h]));
+            acc[n] = fadd2(acc[n], make_float2(fast_exp2(x.x), fast_exp2(x.y)));
+          }
+      float cs[2][2] = {{acc[0].x, acc[0].y}, {acc[1].x, acc[1].y}};
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
 #pragma unroll

@@ -1,15 +1,17 @@
 // attn_sparse.cu -- a sparse-attention layer of a hybrid block (KV Reuse): each query row's
 // own queries attend only to the cache rows its full-attention layer selected, and every
-// gathered K/V row serves all H heads.
+// gathered K/V row serves all query heads of a 16-head group.
 //
 // "HySparse2: How Xiaomi Split the Transformer to Fix Agent Prefill Costs", section "KV Reuse
 // and Token-Level Sparse Selection": the sparse layers take the full layer's indices and cache
 // as they are; the forced-window tokens are ordinary rows of that cache.
 //
-// One CTA per (query row, split of its selected list): warp 4 gathers 64 selected rows per
-// tile with 16-byte cp.async into the swizzled tile layout; warps 0..3 run the same tensor-core
-// online softmax as the full layer. Splits of one row are combined by merge_partials_kernel,
-// which also serves the full layer's decode pass 1.
+// One CTA per (query row, split of the selected list): every warp gathers its share of each
+// 64-row tile (16-byte cp.async into the swizzled tile layout, two stages) and runs the
+// tensor-core online softmax on 16 heads x 16 rows of it. A row's splits write per-warp
+// partials that merge_partials_kernel combines; a row handled by one CTA is merged in
+// shared memory and written directly.
+// merge_partials_kernel (one CTA per output group and head) serves the decode full layer.
 #include "attn_pipeline.cuh"
 #include "internal.h"
 
@@ -17,104 +19,165 @@ namespace hs2 {
 
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-
-
-// Where a CTA's result goes. A group is the set of CTAs that share one output block (a
-// sequence's items in pass 1, a query row's splits in a sparse layer). With one CTA per group
-// the CTA writes the output directly; otherwise it writes its partial (max, denominator,
-// unnormalised output per head) and merge_partials_kernel combines the group afterwards.
-struct MergeTarget {
-  int n_group;
-  float *group_part;   // [n_group][H][kPartRow]
-  int slot;            // this CTA's index in the group
-  void *out;           // [H][128] block of the output
-  int out_f32;
-  float *lse;          // [H] or null
+// One CTA per (query row, split of its selected list), no dedicated producer: the 4 * HG
+// warps each gather 64 / (4 * HG) rows of every tile with 16-byte cp.async (so the copies are
+// issued from all four SM sub-partitions at once) and each computes 16 heads x 16 rows of it.
+template <int KV, int HG>
+struct SpCfg {
+  static constexpr int kWarps = 4 * HG;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kRowsPerWarp = kTile / kWarps;
+  static constexpr int kKBytes = (KV == kKvBf16) ? 2 * kBoxBytes : kBoxBytes;
+  static constexpr int kStageBytes = (2 * kKBytes + (KV == kKvFp8 ? 512 : 0) + 1023) / 1024 * 1024;
+  static constexpr int kStages = 2;
+  // the stage ring doubles as the warp-merge area of a row handled by one CTA
+  static constexpr size_t kMergeBytes = (size_t)kWarps * 16 * (kHeadDim + 2) * 4;
+  static constexpr size_t kRegion = ((size_t)kStages * kStageBytes > kMergeBytes)
+                                        ? (size_t)kStages * kStageBytes : (kMergeBytes + 1023) / 1024 * 1024;
+  static constexpr size_t kSmem = 1024 + kRegion + 2 * kStages * 8 + 16;
 };
 
-// Merges the warps' softmax states (stashed in smem) and delivers the result.
+constexpr int kPreTiles = 24;   // tiles whose indices are fetched up front
+
+// This warp's share of tile `it`: rows [w * RPW, (w+1) * RPW), cp.async into stage `st`, then
+// one arrival per lane on `bar` once the copies land (entries past the list are zero-filled).
 template <int KV, int HG>
-__device__ void finish_cta(const float *ws_o, const float *ws_ml, const MergeTarget &mt) {
-  constexpr int H = 16 * HG;
-  constexpr int TG = kConsumerWarps / HG;
-  const bool direct = mt.n_group == 1;
-  float *part = mt.group_part + (size_t)mt.slot * H * kPartRow;
-  for (int t = threadIdx.x; t < H * kHeadDim; t += kThreads) {
-    const int h = t / kHeadDim, d = t % kHeadDim;
-    const int hg = h >> 4, r = h & 15;
-    float M = -INFINITY;
-    for (int tg = 0; tg < TG; ++tg) M = fmaxf(M, ws_ml[((tg * HG + hg) * 16 + r) * 2]);
-    float L = 0.f, O = 0.f;
-    for (int tg = 0; tg < TG; ++tg) {
-      const int w = tg * HG + hg;
-      const float m = ws_ml[(w * 16 + r) * 2];
-      const float f = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
-      L += f * ws_ml[(w * 16 + r) * 2 + 1];
-      O += f * ws_o[(w * 16 + r) * kHeadDim + d];
+__device__ __forceinline__ void gather_rows(const SparseParams &P, int64_t seq_row0, int64_t p,
+                                            int e_first, int cnt, int warp, uint8_t *st,
+                                            uint32_t bar, int32_t pos_lane, bool &bad) {
+  using C = SpCfg<KV, HG>;
+  const int lane = threadIdx.x & 31;
+  constexpr int RPW = C::kRowsPerWarp;
+  constexpr int CH = (KV == kKvBf16) ? 16 : 8;        // 16-byte chunks per row
+  constexpr int PER = RPW * CH * 2 / 32;               // copies per lane (K and V)
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int q = k * 32 + lane;                       // (row, chunk, K/V) flattened
+    const int kv = q / (RPW * CH);
+    const int rem = q % (RPW * CH);
+    const int rl = rem / CH, ch = rem % CH;
+    const int rr = warp * RPW + rl;
+    const int e = e_first + rr;
+    const bool v = e < cnt;
+    int64_t pos = __shfl_sync(0xffffffffu, pos_lane, rl);
+    if (!v) pos = 0;
+    if (pos < 0 || pos > p) {
+      bad = true;
+      pos = 0;
     }
-    if (direct) {
-      const float val = O / L;
-      if (mt.out_f32) reinterpret_cast<float *>(mt.out)[t] = val;
-      else reinterpret_cast<__nv_bfloat16 *>(mt.out)[t] = __float2bfloat16_rn(val);
-      if (mt.lse && d == 0) mt.lse[h] = (M + __log2f(L)) * kLn2;
+    const int64_t row = seq_row0 + pos;
+    const uint32_t nb = v ? 16u : 0u;
+    if (KV == kKvBf16) {
+      const uint8_t *src = reinterpret_cast<const uint8_t *>(kv ? P.v : P.k) + row * 256 + ch * 16;
+      cp_async_16(smem_u32(st + kv * C::kKBytes + tile_off(kTile, rr, ch * 8)), src, nb);
     } else {
-      part[h * kPartRow + kPartO + d] = O;
-      if (d == 0) {
-        part[h * kPartRow] = M;
-        part[h * kPartRow + 1] = L;
-      }
+      const uint8_t *src = reinterpret_cast<const uint8_t *>(kv ? P.v : P.k) + row * 128 + ch * 16;
+      cp_async_16(smem_u32(st + kv * C::kKBytes + fp8_off(rr, ch * 16)), src, nb);
     }
   }
+  if (KV == kKvFp8 && lane < RPW) {
+    const int rr = warp * RPW + lane;
+    const bool v = e_first + rr < cnt;
+    int64_t pos = v ? pos_lane : 0;
+    if (pos < 0 || pos > p) pos = 0;
+    const int64_t row = seq_row0 + pos;
+    uint8_t *sc = st + 2 * C::kKBytes;
+    cp_async_4(smem_u32(sc + rr * 4), P.k_scale + row, v ? 4u : 0u);
+    cp_async_4(smem_u32(sc + (kTile + rr) * 4), P.v_scale + row, v ? 4u : 0u);
+  }
+  cp_async_mbar_arrive(bar);
 }
 
-// Consumer warps of pass 1 / sparse layers. Warp (hg, tg): heads [16 hg, 16 hg + 16), tile
-// rows [tg * NTW, (tg+1) * NTW) with NTW = 16 * HG. `is_valid(it, rr)` says whether row rr
-// of tile it holds a cache row this CTA attends to. The warp's state is stashed into
-// ws_o / ws_ml (stage memory) at the end.
-template <int KV, int HG, class Valid>
-__device__ void consume_pv(const Valid &is_valid, uint8_t *stages, uint64_t *full,
-                           uint64_t *empty, uint8_t *q_smem, const __nv_bfloat16 *qg,
-                           float scale_log2, int n_tiles, volatile int *abort_flag,
-                           uint32_t *status) {
-  using C = DecodeCfg<KV, 0>;
+template <int KV, int HG>
+__global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads) sparse_gather_kernel(const __grid_constant__ SparseParams P) {
+  using C = SpCfg<KV, HG>;
   constexpr int H = 16 * HG;
-  constexpr int NTW = 16 * HG;
-  constexpr int NT = NTW / 8;
+  constexpr int TG = 4;   // token groups: warp w covers rows [16 * (w / HG), +16) of a tile
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *stages = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(stages + C::kRegion);
+  uint64_t *empty = full + C::kStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + C::kStages);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x / P.n_tsplit, ts = blockIdx.x % P.n_tsplit;
+  const int b = r / P.n_q, i = r % P.n_q;
+  const int64_t seq_row0 = P.seq.start[b];
+  const int64_t p = (int64_t)P.seq.len[b] - P.n_q + i;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(smem_u32(&full[s]), C::kThreads);
+      mbar_init(smem_u32(&empty[s]), C::kWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  griddep_launch_dependents();
+  griddep_wait();   // idx / count come from the selection kernel
+  const int e_begin = ts * P.split_len;
+  // this warp's row indices for its first kPreTiles tiles, fetched together with the count
+  const int32_t *idx = P.idx + (size_t)r * P.idx_stride;
+  int32_t pre[kPreTiles];
+#pragma unroll
+  for (int k = 0; k < kPreTiles; ++k) {
+    const int e = e_begin + k * kTile + warp * C::kRowsPerWarp + lane;
+    pre[k] = (lane < C::kRowsPerWarp && k * kTile < P.split_len && e < P.idx_stride) ? __ldcg(idx + e) : 0;
+  }
+  int cnt = __ldcg(P.count + r);
+  if (cnt < 1 || cnt > P.idx_stride) {
+    if (threadIdx.x == 0) record_status(P.status, kStatusCheck);
+    cnt = max(1, min(cnt, P.idx_stride));
+  }
+  const int n_tiles = max(0, min(P.split_len, cnt - e_begin) + kTile - 1) / kTile;
+  auto pos_of = [&](int it) -> int32_t {
+    int32_t v = 0;
+#pragma unroll
+    for (int k = 0; k < kPreTiles; ++k)
+      if (k == it) v = pre[k];
+    if (it >= kPreTiles) {
+      const int e = e_begin + it * kTile + warp * C::kRowsPerWarp + lane;
+      v = (lane < C::kRowsPerWarp && e < cnt) ? __ldcg(idx + e) : 0;
+    }
+    return v;
+  };
+  bool bad = false;
+  for (int it = 0; it < min(n_tiles, C::kStages); ++it)
+    gather_rows<KV, HG>(P, seq_row0, p, e_begin + it * kTile, cnt, warp, stages + it * C::kStageBytes,
+                        smem_u32(&full[it]), pos_of(it), bad);
+
   const int hg = warp % HG, tg = warp / HG;
-  const int tok0 = tg * NTW;
-  const int g = lane >> 2, c = lane & 3;
+  const int tok0 = tg * 16;
+  const int c = lane & 3, g = lane >> 2;
+  const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(P.q) + (size_t)r * H * kHeadDim;
   uint32_t qa[8][4];
   float rowf[2];
   if (KV == kKvBf16) {
-    load_q_frags_bf16(smem_u32(q_smem), H, hg * 16, qa);
-    rowf[0] = rowf[1] = scale_log2;
+    load_q_frags_bf16_global(qg, hg * 16, qa);
+    rowf[0] = rowf[1] = P.scale_log2;
   } else {
     float pw[2];
     load_q_frags_f16(qg, hg * 16, qa, pw);
-    rowf[0] = scale_log2 * pw[0];
-    rowf[1] = scale_log2 * pw[1];
+    rowf[0] = P.scale_log2 * pw[0];
+    rowf[1] = P.scale_log2 * pw[1];
   }
   WarpSoftmax st;
   st.init();
   for (int it = 0; it < n_tiles; ++it) {
     const int s = it % C::kStages;
     if (!mbar_wait(smem_u32(&full[s]), (it / C::kStages) & 1)) {
-      record_status(status, kStatusTimeout);
+      record_status(P.status, kStatusTimeout);
       *abort_flag = 1;
     }
     if (*abort_flag) break;
     const uint8_t *stg = stages + s * C::kStageBytes;
-    bool valid[NT][2];
-    float colk[NT][2], colv[NT][2];
+    bool valid[2][2];
+    float colk[2][2], colv[2][2];
 #pragma unroll
-    for (int n = 0; n < NT; ++n)
+    for (int n = 0; n < 2; ++n)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int rr = tok0 + n * 8 + 2 * c + e;
-        valid[n][e] = is_valid(it, rr);
+        valid[n][e] = e_begin + it * kTile + rr < cnt;
         if (KV == kKvFp8) {
           const float *sc = reinterpret_cast<const float *>(stg + 2 * C::kKBytes);
           colk[n][e] = sc[rr];
@@ -124,274 +187,83 @@ __device__ void consume_pv(const Valid &is_valid, uint8_t *stages, uint64_t *ful
           colv[n][e] = 1.f;
         }
       }
-    float sacc[NT][4];
-    qk_tile<KV, NT>(qa, smem_u32(stg), tok0, sacc);
-    softmax_pv_tile<KV, NT>(st, sacc, rowf, colk, colv, valid, smem_u32(stg + C::kKBytes), tok0);
+    float sacc[2][4];
+    qk_tile<KV, 2>(qa, smem_u32(stg), tok0, sacc);
+    softmax_pv_tile<KV, 2>(st, sacc, rowf, colk, colv, valid, smem_u32(stg + C::kKBytes), tok0);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+    const int nxt = it + C::kStages;
+    if (nxt < n_tiles) {   // refill this stage once every warp is done with it
+      if (!mbar_wait(smem_u32(&empty[s]), (it / C::kStages) & 1)) {
+        record_status(P.status, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      gather_rows<KV, HG>(P, seq_row0, p, e_begin + nxt * kTile, cnt, warp, stages + s * C::kStageBytes,
+                          smem_u32(&full[s]), pos_of(nxt), bad);
+    }
   }
+  if (bad) record_status(P.status, kStatusCheck);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     st.l[h] += __shfl_xor_sync(0xffffffffu, st.l[h], 1);
     st.l[h] += __shfl_xor_sync(0xffffffffu, st.l[h], 2);
   }
-  // every consumer is done with the stages before they are reused for the merge
-  named_barrier_sync(1, kConsumerWarps * 32);
-  float *ws_o = reinterpret_cast<float *>(stages);              // [warp][16][128]
-  float *ws_ml = ws_o + kConsumerWarps * 16 * kHeadDim;         // [warp][16][2]
+  if (P.n_tsplit > 1) {
+    // this warp's partial: slot ts * TG + tg of row r, its 16 heads (combined by the merge kernel)
+    const int slot = ts * TG + tg;
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float *row = P.part + (((size_t)r * P.n_tsplit * TG + slot) * H + hg * 16 + g + 8 * hh) * kPartRow;
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) row[kPartO + o_col<KV>(n, e, c)] = st.o[n][2 * hh + e] * st.vref;
+      if (c == 0) {
+        row[0] = st.m[hh];
+        row[1] = st.l[hh];
+      }
+    }
+    return;
+  }
+  // one CTA per row: merge the token groups through shared memory (stages are free once every
+  // warp is past its last tile)
+  __syncthreads();
+  if (*abort_flag) return;
+  float *ws_o = reinterpret_cast<float *>(stages);      // [warp][16][128]
+  float *ws_ml = ws_o + C::kWarps * 16 * kHeadDim;      // [warp][16][2]
 #pragma unroll
   for (int n = 0; n < 16; ++n)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int r = g + (e >> 1) * 8;
-      ws_o[(warp * 16 + r) * kHeadDim + o_col<KV>(n, e & 1, c)] = st.o[n][e] * st.vref;
-    }
+    for (int e = 0; e < 4; ++e)
+      ws_o[(warp * 16 + g + (e >> 1) * 8) * kHeadDim + o_col<KV>(n, e & 1, c)] = st.o[n][e] * st.vref;
   if (c == 0) {
     ws_ml[(warp * 16 + g) * 2 + 0] = st.m[0];
     ws_ml[(warp * 16 + g) * 2 + 1] = st.l[0];
     ws_ml[(warp * 16 + g + 8) * 2 + 0] = st.m[1];
     ws_ml[(warp * 16 + g + 8) * 2 + 1] = st.l[1];
   }
-}
-
-// Shared memory of a pass-1 / sparse CTA: stages | Q (bf16, H rows) | barriers | abort flag
-template <int KV, int HG>
-struct PvSmem {
-  using C = DecodeCfg<KV, 0>;
-  uint8_t *stages, *q;
-  uint64_t *full, *empty;
-  volatile int *abort_flag;
-  __device__ explicit PvSmem(uint8_t *raw) {
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-    stages = base;
-    q = stages + C::kStages * C::kStageBytes;
-    full = reinterpret_cast<uint64_t *>(q + 16 * HG * 256);
-    empty = full + C::kStages;
-    abort_flag = reinterpret_cast<volatile int *>(empty + C::kStages);
-  }
-  static constexpr size_t bytes() {
-    return 1024 + C::kStages * C::kStageBytes + 16 * HG * 256 + 2 * C::kStages * 8 + 16;
-  }
-};
-
-template <int HG>
-__device__ __forceinline__ void stage_q_bf16(uint8_t *q_smem, const __nv_bfloat16 *qg) {
-  constexpr int H = 16 * HG;
-  for (int t = threadIdx.x; t < H * 16; t += kThreads) {
-    const int r = t >> 4, ch = t & 15;
-    const uint4 v = *reinterpret_cast<const uint4 *>(qg + r * kHeadDim + ch * 8);
-    *reinterpret_cast<uint4 *>(q_smem + tile_off(H, r, ch * 8)) = v;
-  }
-}
-
-// Sparse layer: gather producer. All 32 lanes of the producer warp copy two gathered rows
-// each per tile with 16-byte cp.async, then arrive on the stage's barrier when they land.
-template <int KV>
-__device__ void produce_gather(const SparseParams &P, int r, int64_t seq_row0, int64_t p,
-                               int e_begin, int cnt, uint8_t *stages, uint64_t *full,
-                               uint64_t *empty, int n_tiles, volatile int *abort_flag) {
-  using C = DecodeCfg<KV, 0>;
-  const int lane = threadIdx.x & 31;
-  const int32_t *idx = P.idx + (size_t)r * P.idx_stride;
-  bool bad = false;
-  for (int it = 0; it < n_tiles; ++it) {
-    const int s = it % C::kStages;
-    const uint32_t par = ((it / C::kStages) & 1) ^ 1;
-    if (it >= C::kStages) {
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), par);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        if (lane == 0) {
-          record_status(P.status, kStatusTimeout);
-          *abort_flag = 1;
-        }
-        return;
-      }
-    }
-    if (*abort_flag) return;
-    uint8_t *st = stages + s * C::kStageBytes;
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int rr = 2 * lane + u;
-      const int e = e_begin + it * kTile + rr;
-      const bool v = e < cnt;
-      int64_t pos = v ? (int64_t)__ldcg(idx + e) : 0;
-      if (pos < 0 || pos > p) {   // out-of-range index: flag it and read row 0 instead
-        bad = true;
-        pos = 0;
-      }
-      const int64_t row = seq_row0 + pos;
-      const uint32_t nb = v ? 16u : 0u;
-      if (KV == kKvBf16) {
-        const uint8_t *ksrc = reinterpret_cast<const uint8_t *>(P.k) + row * 256;
-        const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(P.v) + row * 256;
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          cp_async_16(smem_u32(st + tile_off(kTile, rr, ch * 8)), ksrc + ch * 16, nb);
-          cp_async_16(smem_u32(st + C::kKBytes + tile_off(kTile, rr, ch * 8)), vsrc + ch * 16, nb);
-        }
-      } else {
-        const uint8_t *ksrc = reinterpret_cast<const uint8_t *>(P.k) + row * 128;
-        const uint8_t *vsrc = reinterpret_cast<const uint8_t *>(P.v) + row * 128;
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          cp_async_16(smem_u32(st + fp8_off(rr, ch * 16)), ksrc + ch * 16, nb);
-          cp_async_16(smem_u32(st + C::kKBytes + fp8_off(rr, ch * 16)), vsrc + ch * 16, nb);
-        }
-        uint8_t *sc = st + 2 * C::kKBytes;
-        cp_async_4(smem_u32(sc + rr * 4), P.k_scale + row, v ? 4u : 0u);
-        cp_async_4(smem_u32(sc + (kTile + rr) * 4), P.v_scale + row, v ? 4u : 0u);
-      }
-    }
-    cp_async_mbar_arrive(smem_u32(&full[s]));
-  }
-  if (bad) record_status(P.status, kStatusCheck);
-}
-
-struct CountValid {
-  int e_begin, cnt;
-  __device__ bool operator()(int it, int rr) const { return e_begin + it * kTile + rr < cnt; }
-};
-
-template <int KV, int HG>
-__global__ void __launch_bounds__(kThreads, 1) sparse_gather_kernel(const __grid_constant__ SparseParams P) {
-  using C = DecodeCfg<KV, 0>;
-  constexpr int H = 16 * HG;
-  constexpr int NTW = 16 * HG;             // rows of a tile per warp
-  constexpr int NT = NTW / 8;
-  constexpr int TG = kConsumerWarps / HG;  // token groups per CTA
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  PvSmem<KV, HG> sm(smem_raw);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x / P.n_split, j = blockIdx.x % P.n_split;
-  const int b = r / P.n_q, i = r % P.n_q;
-  const int64_t seq_row0 = P.seq.start[b];
-  const int64_t p = (int64_t)P.seq.len[b] - P.n_q + i;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(smem_u32(&sm.full[s]), 32);
-      mbar_init(smem_u32(&sm.empty[s]), kConsumerWarps);
-    }
-    *sm.abort_flag = 0;
-    fence_barrier_init();
-  }
   __syncthreads();
-  griddep_launch_dependents();
-  griddep_wait();   // idx / count come from the selection kernel
-  int cnt = __ldcg(P.count + r);
-  if (cnt < 1 || cnt > P.idx_stride) {
-    if (threadIdx.x == 0) record_status(P.status, kStatusCheck);
-    cnt = max(1, min(cnt, P.idx_stride));
+  for (int t = threadIdx.x; t < H * kHeadDim; t += C::kThreads) {
+    const int h = t / kHeadDim, d = t % kHeadDim;
+    const int hgh = h >> 4, rh = h & 15;
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < TG; ++k) M = fmaxf(M, ws_ml[((k * HG + hgh) * 16 + rh) * 2]);
+    float L = 0.f, O = 0.f;
+#pragma unroll
+    for (int k = 0; k < TG; ++k) {
+      const int w = k * HG + hgh;
+      const float m = ws_ml[(w * 16 + rh) * 2];
+      const float f = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
+      L += f * ws_ml[(w * 16 + rh) * 2 + 1];
+      O += f * ws_o[(w * 16 + rh) * kHeadDim + d];
+    }
+    const float val = O / L;
+    const size_t oi = ((size_t)r * H + h) * kHeadDim + d;
+    if (P.out_f32) reinterpret_cast<float *>(P.out)[oi] = val;
+    else reinterpret_cast<__nv_bfloat16 *>(P.out)[oi] = __float2bfloat16_rn(val);
   }
-  const int e_begin = j * P.split_len;
-  const int n_tiles = max(0, min(P.split_len, cnt - e_begin) + kTile - 1) / kTile;
-  const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(P.q) + (size_t)r * H * kHeadDim;
-  WarpSoftmax st;
-  st.init();
-  const int hg = warp % HG, tg = warp / HG;
-  if (warp == kConsumerWarps) {
-    produce_gather<KV>(P, r, seq_row0, p, e_begin, cnt, sm.stages, sm.full, sm.empty, n_tiles,
-                       sm.abort_flag);
-  } else {
-    const int tok0 = tg * NTW;
-    const int c = lane & 3;
-    uint32_t qa[8][4];
-    float rowf[2];
-    if (KV == kKvBf16) {
-      load_q_frags_bf16_global(qg, hg * 16, qa);
-      rowf[0] = rowf[1] = P.scale_log2;
-    } else {
-      float pw[2];
-      load_q_frags_f16(qg, hg * 16, qa, pw);
-      rowf[0] = P.scale_log2 * pw[0];
-      rowf[1] = P.scale_log2 * pw[1];
-    }
-    for (int it = 0; it < n_tiles; ++it) {
-      const int s = it % C::kStages;
-      if (!mbar_wait(smem_u32(&sm.full[s]), (it / C::kStages) & 1)) {
-        record_status(P.status, kStatusTimeout);
-        *sm.abort_flag = 1;
-      }
-      if (*sm.abort_flag) break;
-      const uint8_t *stg = sm.stages + s * C::kStageBytes;
-      bool valid[NT][2];
-      float colk[NT][2], colv[NT][2];
-#pragma unroll
-      for (int n = 0; n < NT; ++n)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int rr = tok0 + n * 8 + 2 * c + e;
-          valid[n][e] = e_begin + it * kTile + rr < cnt;
-          if (KV == kKvFp8) {
-            const float *sc = reinterpret_cast<const float *>(stg + 2 * C::kKBytes);
-            colk[n][e] = sc[rr];
-            colv[n][e] = sc[kTile + rr];
-          } else {
-            colk[n][e] = 1.f;
-            colv[n][e] = 1.f;
-          }
-        }
-      float sacc[NT][4];
-      qk_tile<KV, NT>(qa, smem_u32(stg), tok0, sacc);
-      softmax_pv_tile<KV, NT>(st, sacc, rowf, colk, colv, valid, smem_u32(stg + C::kKBytes), tok0);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      st.l[h] += __shfl_xor_sync(0xffffffffu, st.l[h], 1);
-      st.l[h] += __shfl_xor_sync(0xffffffffu, st.l[h], 2);
-    }
-    if (P.n_split > 1) {
-      // this warp's partial: slot j * TG + tg of row r, its 16 heads
-      const int g = lane >> 2;
-      const int slot = j * TG + tg;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float *row = P.part + (((size_t)r * P.n_split * TG + slot) * H + hg * 16 + g + 8 * hh) * kPartRow;
-#pragma unroll
-        for (int n = 0; n < 16; ++n)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) row[kPartO + o_col<KV>(n, e, c)] = st.o[n][2 * hh + e] * st.vref;
-        if (c == 0) {
-          row[0] = st.m[hh];
-          row[1] = st.l[hh];
-        }
-      }
-    } else {
-      // one CTA per row: merge the token groups through shared memory (stages are free once
-      // every consumer has finished its tiles)
-      named_barrier_sync(1, kConsumerWarps * 32);
-      float *ws_o = reinterpret_cast<float *>(sm.stages);
-      float *ws_ml = ws_o + kConsumerWarps * 16 * kHeadDim;
-      const int g = lane >> 2;
-#pragma unroll
-      for (int n = 0; n < 16; ++n)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          ws_o[(warp * 16 + g + (e >> 1) * 8) * kHeadDim + o_col<KV>(n, e & 1, c)] = st.o[n][e] * st.vref;
-      if (c == 0) {
-        ws_ml[(warp * 16 + g) * 2 + 0] = st.m[0];
-        ws_ml[(warp * 16 + g) * 2 + 1] = st.l[0];
-        ws_ml[(warp * 16 + g + 8) * 2 + 0] = st.m[1];
-        ws_ml[(warp * 16 + g + 8) * 2 + 1] = st.l[1];
-      }
-    }
-  }
-  if (P.n_split > 1) return;
-  __syncthreads();
-  if (*sm.abort_flag) return;
-  const float *ws_o = reinterpret_cast<const float *>(sm.stages);
-  MergeTarget mt;
-  mt.n_group = 1;
-  mt.group_part = nullptr;
-  mt.slot = 0;
-  mt.out_f32 = P.out_f32;
-  mt.out = P.out_f32 ? (void *)(reinterpret_cast<float *>(P.out) + (size_t)r * H * kHeadDim)
-                     : (void *)(reinterpret_cast<__nv_bfloat16 *>(P.out) + (size_t)r * H * kHeadDim);
-  mt.lse = nullptr;
-  finish_cta<KV, HG>(ws_o, ws_o + kConsumerWarps * 16 * kHeadDim, mt);
 }
 
 // One CTA per (group, head): 8 slot lanes x 32 lanes of 4 output dims; float4 loads.
@@ -468,18 +340,14 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __g
 }
 
 template <int KV, int HG>
-constexpr size_t sparse_smem() {
-  return PvSmem<KV, HG>::bytes();
-}
-
-template <int KV, int HG>
 cudaError_t launch_sparse_t(const SparseParams &p, cudaStream_t s) {
-  const size_t smem = sparse_smem<KV, HG>();
+  using C = SpCfg<KV, HG>;
+  static_assert(C::kSmem <= 227 * 1024, "sparse shared memory");
   auto kern = sparse_gather_kernel<KV, HG>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (e != cudaSuccess) return e;
-  const int grid = p.batch * p.n_q * p.n_split;
-  e = launch_pdl(kern, grid, kThreads, smem, s, p);
+  const int grid = p.batch * p.n_q * p.n_tsplit;
+  e = launch_pdl(kern, grid, C::kThreads, C::kSmem, s, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

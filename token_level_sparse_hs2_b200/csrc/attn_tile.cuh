@@ -66,6 +66,25 @@ __device__ __forceinline__ uint32_t fp8_off(int r, int b) {
   return r * 128 + ((((b >> 4)) ^ (r & 7)) << 4) + (b & 15);
 }
 
+// Tile layouts. kSwz: TMA tiles with the 128-byte swizzle (tile_off / fp8_off). kPad: rows
+// copied one by one (bulk copies) at a padded stride of 272 B (bf16) or 144 B (e4m3) -- 16
+// bytes past the row, which spreads the 8 rows of an ldmatrix over distinct bank groups.
+enum TileLayout { kSwz = 0, kPad = 1 };
+constexpr int kPadRowBf16 = 272;
+constexpr int kPadRowFp8 = 144;
+
+template <int LAYOUT>
+__device__ __forceinline__ uint32_t bf16_at(int r, int d) {
+  if (LAYOUT == kSwz) return tile_off(kTile, r, d);
+  return r * kPadRowBf16 + d * 2;
+}
+
+template <int LAYOUT>
+__device__ __forceinline__ uint32_t fp8_at(int r, int b) {
+  if (LAYOUT == kSwz) return fp8_off(r, b);
+  return r * kPadRowFp8 + b;
+}
+
 // head_dim column of output fragment (n8 tile n, column element e&1) for lane c
 template <int KV>
 __device__ __forceinline__ int o_col(int n, int ecol, int c) {
@@ -135,7 +154,7 @@ __device__ __forceinline__ void load_q_frags_f16(const __nv_bfloat16 *q, int row
 
 // ------------------------------------------------------------------ S = Q . K^T
 
-template <int KV, int NT>
+template <int KV, int NT, int LAYOUT = kSwz>
 __device__ __forceinline__ void qk_tile(const uint32_t (&qa)[8][4], uint32_t k_smem, int tok0,
                                         float (&s)[NT][4]) {
   const int lane = threadIdx.x & 31;
@@ -152,7 +171,7 @@ __device__ __forceinline__ void qk_tile(const uint32_t (&qa)[8][4], uint32_t k_s
         const int r = tok0 + np * 16 + (i >> 1) * 8 + j;
         const int d = ks * 16 + (i & 1) * 8;
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(k_smem + tile_off(kTile, r, d), b0, b1, b2, b3);
+        ldsm_x4(k_smem + bf16_at<LAYOUT>(r, d), b0, b1, b2, b3);
         mma_bf16(s[2 * np], qa[ks], b0, b1);
         mma_bf16(s[2 * np + 1], qa[ks], b2, b3);
       }
@@ -166,7 +185,7 @@ __device__ __forceinline__ void qk_tile(const uint32_t (&qa)[8][4], uint32_t k_s
         const int r = tok0 + n * 8 + j;
         const int kb = 4 * half + i;
         uint32_t w[4];
-        ldsm_x4(k_smem + fp8_off(r, kb * 16), w[0], w[1], w[2], w[3]);
+        ldsm_x4(k_smem + fp8_at<LAYOUT>(r, kb * 16), w[0], w[1], w[2], w[3]);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint32_t b0 = e4m3x2_to_f16x2(w[q] & 0xffffu);
@@ -178,9 +197,78 @@ __device__ __forceinline__ void qk_tile(const uint32_t (&qa)[8][4], uint32_t k_s
   }
 }
 
+// S[mt] = Q[mt] . K^T for MT m-tiles (16 heads each) sharing every K fragment: each fragment
+// is loaded (and, for e4m3, widened) once and fed to all MT tensor-core products.
+template <int KV, int MT, int NT, int LAYOUT = kSwz>
+__device__ __forceinline__ void qk_tile_mt(const uint32_t (&qa)[MT][8][4], uint32_t k_smem,
+                                           int tok0, float (&s)[MT][NT][4]) {
+  const int lane = threadIdx.x & 31;
+  const int i = lane >> 3, j = lane & 7;
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[m][n][e] = 0.f;
+  if (KV == kKvBf16) {
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        const int r = tok0 + np * 16 + (i >> 1) * 8 + j;
+        const int d = ks * 16 + (i & 1) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(k_smem + bf16_at<LAYOUT>(r, d), b0, b1, b2, b3);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          mma_bf16(s[m][2 * np], qa[m][ks], b0, b1);
+          mma_bf16(s[m][2 * np + 1], qa[m][ks], b2, b3);
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int r = tok0 + n * 8 + j;
+        const int kb = 4 * half + i;
+        uint32_t w[4];
+        ldsm_x4(k_smem + fp8_at<LAYOUT>(r, kb * 16), w[0], w[1], w[2], w[3]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t b0 = e4m3x2_to_f16x2(w[q] & 0xffffu);
+          const uint32_t b1 = e4m3x2_to_f16x2(w[q] >> 16);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) mma_f16(s[m][n], qa[m][4 * half + q], b0, b1);
+        }
+      }
+    }
+  }
+}
+
+// Packed fp32 pair arithmetic (sm_100): two fused multiply-adds / adds per instruction.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // ------------------------------------------------------------------ O += P . V
 
-template <int KV, int NT>
+template <int KV, int NT, int LAYOUT = kSwz>
 __device__ __forceinline__ void pv_tile(const uint32_t (&pa)[NT / 2][4], uint32_t v_smem,
                                         int tok0, float (&o)[16][4]) {
   const int lane = threadIdx.x & 31;
@@ -193,7 +281,7 @@ __device__ __forceinline__ void pv_tile(const uint32_t (&pa)[NT / 2][4], uint32_
         const int r = tok0 + kk * 16 + (i & 1) * 8 + j;
         const int d = dp * 16 + (i >> 1) * 8;
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(v_smem + tile_off(kTile, r, d), b0, b1, b2, b3);
+        ldsm_x4_t(v_smem + bf16_at<LAYOUT>(r, d), b0, b1, b2, b3);
         mma_bf16(o[2 * dp], pa[kk], b0, b1);
         mma_bf16(o[2 * dp + 1], pa[kk], b2, b3);
       }
@@ -204,7 +292,7 @@ __device__ __forceinline__ void pv_tile(const uint32_t (&pa)[NT / 2][4], uint32_
         const int r = tok0 + kk * 16 + (i & 1) * 8 + j;
         const int kb = 2 * kp + (i >> 1);
         uint32_t w[4];
-        ldsm_x4_t(v_smem + fp8_off(r, kb * 16), w[0], w[1], w[2], w[3]);
+        ldsm_x4_t(v_smem + fp8_at<LAYOUT>(r, kb * 16), w[0], w[1], w[2], w[3]);
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
           const uint32_t lo = prmt(w[2 * hb], 0, 0x3120);       // rows 0..7:  (even | odd)
@@ -249,7 +337,7 @@ struct WarpSoftmax {
 // share the reference, and the final log-sum-exp is m + log2(l). For e4m3 caches the V-scale
 // reference st.vref likewise only moves when the tile's largest scale leaves
 // [vref * 2^-8, vref * 2^11], which keeps P * v_scale / vref within f16 range.
-template <int KV, int NT>
+template <int KV, int NT, int LAYOUT = kSwz>
 __device__ __forceinline__ void softmax_pv_tile(WarpSoftmax &st, float (&s)[NT][4],
                                                 const float (&rowf)[2],
                                                 const float (&colk)[NT][2],
@@ -337,7 +425,7 @@ __device__ __forceinline__ void softmax_pv_tile(WarpSoftmax &st, float (&s)[NT][
       st.o[n][3] *= a1;
     }
   }
-  pv_tile<KV, NT>(pa, v_smem, tok0, st.o);
+  pv_tile<KV, NT, LAYOUT>(pa, v_smem, tok0, st.o);
 }
 
 }  // namespace hs2

@@ -154,7 +154,7 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   P.off_hist = o; o = align_up(o + (P.n_seg > 1 ? 4 * (size_t)kHistBins * P.n_rows : 0));
   P.off_cand_count = o; o = align_up(o + 4 * (size_t)P.n_rows);
   P.off_arrive = o; o = align_up(o + 4 * (size_t)P.n_rows);
-  P.off_cnt_sp = o; o = align_up(o + 4 * (size_t)P.n_rows);
+  P.off_cnt_sp = o; o = align_up(o + 4 * (size_t)P.n_rows * (P.H / 16));
   P.zero_end = o;
   const size_t part_row = (size_t)P.H * kPartRow * 4;
   const size_t max_slots =
@@ -165,7 +165,8 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   const size_t cand = (P.n_seg > 1) ? (size_t)P.n_rows * kCandCapGlobal * 4 : 0;
   P.off_cand_key = o; o = align_up(o + cand);
   P.off_cand_idx = o; o = align_up(o + cand);
-  P.off_part_sp = o; o = align_up(o + (P.sparse_split ? part_row * kMaxSplit * 4 * P.n_rows : 0));
+  P.off_part_sp = o;
+  o = align_up(o + (P.sparse_split ? (size_t)P.n_rows * kMaxSplit * 4 * P.H * kPartRow * 4 : 0));
   P.total = o;
 }
 
@@ -482,17 +483,13 @@ hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const
   sp.n_q = P.n_q;
   sp.n_heads = P.H;
   const int64_t cap = std::min<int64_t>(idx_stride, P.max_p + 1);
-  if (P.sparse_split) {
-    const int tiles = (int)((cap + kTile - 1) / kTile);
-    int n_split = std::max(1, std::min(tiles, (kManyRows + P.n_rows - 1) / P.n_rows));
-    n_split = std::min(n_split, kMaxSplit);
-    const int tiles_per = (tiles + n_split - 1) / n_split;
-    sp.split_len = tiles_per * kTile;
-    sp.n_split = (int)((cap + sp.split_len - 1) / sp.split_len);
-  } else {
-    sp.n_split = 1;
-    sp.split_len = (int)(((cap + kTile - 1) / kTile) * kTile);
-  }
+  const int tiles = (int)((cap + kTile - 1) / kTile);
+  int ts = 1;
+  if (P.sparse_split)   // about one CTA per SM: spread the gather over the chip
+    ts = std::max(1, std::min({(kManyRows + P.n_rows - 1) / P.n_rows, tiles, kMaxSplit}));
+  const int tiles_per = (tiles + ts - 1) / ts;
+  sp.split_len = tiles_per * kTile;
+  sp.n_tsplit = (int)((cap + sp.split_len - 1) / sp.split_len);
   sp.scale_log2 = scale * 1.4426950408889634f;
   sp.q = q;
   sp.idx = idx;
@@ -508,12 +505,12 @@ hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const
   sp.counter = ws_at<int32_t>(ws, P.off_cnt_sp);
   sp.status = ws_at<uint32_t>(ws, P.off_status);
   hs2_status st = cuda_check(launch_sparse(P.kv_dtype, sp, stream), "sparse gather attention");
-  if (st != HS2_OK || sp.n_split == 1) return st;
+  if (st != HS2_OK || sp.n_tsplit == 1) return st;
   MergeParams mp;
   memset(&mp, 0, sizeof mp);
   mp.by_seq = 0;
   mp.n_groups = P.n_rows;
-  mp.n_fixed = sp.n_split * (4 / (P.H / 16));   // partial slots per row: splits x token groups
+  mp.n_fixed = sp.n_tsplit * 4;   // per-warp partial slots per row: splits x token groups
   mp.n_heads = P.H;
   mp.part = sp.part;
   mp.out = out;

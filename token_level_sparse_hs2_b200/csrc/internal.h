@@ -88,7 +88,7 @@ struct RowsParams {
 struct SparseParams {
   SeqTable seq;
   int32_t batch, n_q, n_heads;
-  int32_t n_split;          // CTAs per query row
+  int32_t n_tsplit;         // CTAs per row along the selected list
   int32_t split_len;        // selected entries per CTA (multiple of 64)
   float scale_log2;
   const void *q;            // bf16 [B, n_q, H, 128]
@@ -99,8 +99,8 @@ struct SparseParams {
   const float *k_scale, *v_scale;
   void *out;
   int32_t out_f32;
-  float *part;              // [B*n_q, n_split, H, 2 + 128]
-  int32_t *counter;         // [B*n_q]
+  float *part;              // [B*n_q, n_tsplit * 4, H, kPartRow] per-warp partials (n_tsplit > 1)
+  int32_t *counter;         // unused
   uint32_t *status;
 };
 

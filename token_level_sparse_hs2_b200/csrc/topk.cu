@@ -352,6 +352,18 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
   // 1. top-digit histogram
   const uint32_t *gh = P.hist ? P.hist + (size_t)r * kHistBins
                               : (P.hist_ws ? P.hist_ws + (size_t)r * kHistBins : nullptr);
+  const int64_t s0 = (int64_t)sg * P.seg_len, s1 = min(nc, s0 + P.seg_len);
+  // a short segment (the usual split case) is read into registers together with the histogram
+  constexpr int kRegKeys = 32;
+  const bool in_regs = gh && P.seg_len <= kRegKeys * kThreadsTk;
+  uint32_t rk[kRegKeys];
+  if (in_regs) {
+#pragma unroll
+    for (int u = 0; u < kRegKeys; ++u) {
+      const int64_t t = s0 + u * kThreadsTk + threadIdx.x;
+      rk[u] = t < s1 ? load_key(s, t) : 0u;
+    }
+  }
   if (gh) {
     for (int t = threadIdx.x; t < kHistBins; t += kThreadsTk) sm.hist[t] = __ldcg(gh + t);
   } else {   // single segment: build it here
@@ -376,11 +388,18 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
   const int B1 = sm.bucket;
   const uint32_t above = sm.above;
   // 3. compact every candidate of this segment with top digit >= B1
-  const int64_t s0 = (int64_t)sg * P.seg_len, s1 = min(nc, s0 + P.seg_len);
   int32_t *gcount = P.cand_count + r;
   uint32_t *gkey = P.cand_key + (size_t)r * P.cand_cap;
   int32_t *gidx = P.cand_idx + (size_t)r * P.cand_cap;
-  for (int64_t base = s0; base < s1; base += kThreadsTk * kUnroll) {
+  if (in_regs) {
+#pragma unroll
+    for (int u = 0; u < kRegKeys; ++u) {
+      const int64_t t = s0 + u * kThreadsTk + threadIdx.x;
+      const bool take = t < s1 && (int)(rk[u] >> 21) >= B1;
+      append<true>(take, rk[u], (int32_t)t, &sm.n_cand, sm.key, sm.idx, kCandCap);
+    }
+  }
+  for (int64_t base = in_regs ? s1 : s0; base < s1; base += kThreadsTk * kUnroll) {
     uint32_t k[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
