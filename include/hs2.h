@@ -145,9 +145,11 @@ hs2_status hs2_block_decode(const hs2_kv_view *kv, const void *q_full,
 
 /* hs2_block_decode, plus one cudaEvent_t (cast to void *) recorded on `stream` before the
  * first enqueued operation and after each step: events[0] before the workspace clear,
- * events[1] after it, events[2] after full-attention pass 1, events[3] after score pass 2,
- * events[4] after the selection, events[5 + l] after sparse layer l. n_events must be
- * 5 + n_sparse. For timing individual kernels without a profiler; results are identical. */
+ * events[1] after it, events[2] after the full-attention pass 1 kernel, events[3] after the
+ * merge of its partial results (no kernel for chunk/prefill queries, whose pass 1 merges
+ * inside), events[4] after score pass 2, events[5] after the selection, events[6 + l] after
+ * sparse layer l. n_events must be 6 + n_sparse. For timing individual kernels without a
+ * profiler; results are identical. */
 hs2_status hs2_block_decode_traced(const hs2_kv_view *kv, const void *q_full,
                                    const void *const *q_sparse, int32_t n_sparse, int32_t topk,
                                    int32_t window, float softmax_scale, void *out_full,
@@ -188,6 +190,11 @@ hs2_status hs2_read_device_status(const void *workspace, void *stream);
 const char *hs2_last_error(void);
 const char *hs2_status_string(hs2_status status);
 int32_t hs2_version(void);
+
+/* Number of kernels this library has launched in the calling process since it was loaded
+ * (successful launches only; the workspace clears done with cudaMemsetAsync are not counted).
+ * Not part of the method: an accounting aid for callers that count launches per call. */
+uint64_t hs2_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
         L.hs2_status_string.restype = ctypes.c_char_p
         L.hs2_status_string.argtypes = [ctypes.c_int]
         L.hs2_version.restype = I32
+        L.hs2_launch_count.restype = ctypes.c_uint64
         for name in ("hs2_workspace_size", "hs2_full_attn_scores", "hs2_topk_select",
                      "hs2_sparse_gather_attn", "hs2_block_decode", "hs2_block_decode_traced",
                      "hs2_topk_select_noalloc", "hs2_read_device_status"):
@@ -217,9 +218,9 @@ def block_decode_traced(cache: KvCache, q_full, q_sparse: Sequence[torch.Tensor]
                         out_sparse: Sequence[torch.Tensor], lse, scores, idx, count, workspace,
                         events: Sequence[torch.cuda.Event], topk=TOPK, window=WINDOW,
                         scale=None, stream=None):
-    """block_decode that also records `events` (5 + n_sparse torch.cuda.Event) around each
-    step on the launch stream: before the clear, then after clear, pass 1, pass 2, selection
-    and each sparse layer."""
+    """block_decode that also records `events` (6 + n_sparse torch.cuda.Event) around each
+    step on the launch stream: before the clear, then after the clear, the pass 1 kernel, the
+    pass 1 merge, pass 2, the selection and each sparse layer."""
     scale = default_scale() if scale is None else scale
     L = len(q_sparse)
     qs = (ctypes.c_void_p * max(L, 1))(*[t.data_ptr() for t in q_sparse])
@@ -236,3 +237,8 @@ def block_decode_traced(cache: KvCache, q_full, q_sparse: Sequence[torch.Tensor]
 def read_device_status(workspace, stream=None):
     """Synchronises and raises HS2Error if a kernel of the last call recorded a problem."""
     _check(lib().hs2_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process so far (hs2_launch_count)."""
+    return int(lib().hs2_launch_count())

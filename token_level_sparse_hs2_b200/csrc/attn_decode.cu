@@ -41,8 +41,11 @@ struct StreamCfg {
   static constexpr int kStages = (KV == kKvBf16) ? (PASS == 0 ? 5 : 4) : (PASS == 0 ? 8 : 6);
   static constexpr uint32_t kTxBytes = kKBytes + kVBytes;
   static constexpr uint32_t kFullCount = (KV == kKvFp8) ? 33 : 1;
+  // pass 1: the consumer warps' partials of a sequence merge in shared memory ([H][128] output
+  // sums, then [8 warps][16 rows] max and denominator) before one partial per CTA is written
+  static constexpr size_t kMergeBytes = (PASS == 0) ? (size_t)16 * HG * o_stride<KV>() * 4 + 8 * 16 * 2 * 4 : 0;
   static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 2 * kStages * 8 + 16 +
-                                  (PASS == 1 ? 2 * (size_t)kHistBins * 4 : 0);
+                                  (PASS == 1 ? 2 * (size_t)kHistBins * 4 : 0) + kMergeBytes;
 };
 
 __device__ __forceinline__ int seq_of_tile(const SeqTable &t, int batch, int g) {
@@ -154,6 +157,7 @@ struct StreamSmem {
   uint64_t *full, *empty;
   volatile int *abort_flag;
   uint32_t *hist;
+  float *merge_o, *merge_ml;
   __device__ explicit StreamSmem(uint8_t *raw) {
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     stages = base;
@@ -161,6 +165,8 @@ struct StreamSmem {
     empty = full + C::kStages;
     abort_flag = reinterpret_cast<volatile int *>(empty + C::kStages);
     hist = reinterpret_cast<uint32_t *>(empty + C::kStages + 2);
+    merge_o = reinterpret_cast<float *>(empty + C::kStages + 2 + (PASS == 1 ? kHistBins : 0));
+    merge_ml = merge_o + (PASS == 0 ? 16 * HG * o_stride<KV>() : 0);
   }
 };
 
@@ -180,33 +186,65 @@ __device__ __forceinline__ void load_q_rows(const __nv_bfloat16 *q, int row0, ui
 
 // ------------------------------------------------------------------ pass 1
 
-// A consumer warp's partial for sequence b: slot = first slot of b + (CTA - first CTA of b) *
-// decode_slots_per_cta(H) + the warp's token group (over all groups); rows are its 16 heads.
+// The CTA's partial for sequence b, written at slot = first slot of b + (CTA - first CTA of b).
+// All consumer warps reach every flush together (they walk the same steps); they exchange their
+// row maxima, add their outputs rescaled to the common maximum into shared memory in a fixed
+// warp order (so results are bitwise reproducible), and the sum is written out once. Named
+// barrier 1 spans the consumer warps only.
 template <int KV, int HG>
-__device__ __forceinline__ void flush_partial(const DecodeParams &P, int b, int tg, int hg,
-                                              const WarpSoftmax &st) {
+__device__ void flush_partial(const DecodeParams &P, int b, int hg, const WarpSoftmax &st,
+                              float *mo, float *mml) {
+  using C = StreamCfg<KV, HG, 0>;
   constexpr int H = 16 * HG;
-  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int first = cta_of_tile(P.seq.tile_begin[b], gridDim.x, P.total_tiles);
-  const int slot = P.seq.item_begin[b] + (blockIdx.x - first) * decode_slots_per_cta(H) + tg;
+  constexpr int NT = C::kConsumers * 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
   float l[2] = {st.l[0], st.l[1]};
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
     l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
   }
+  if (c == 0) {
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    float *row = P.part + ((size_t)slot * H + hg * 16 + g + 8 * hh) * kPartRow;
-#pragma unroll
-    for (int n = 0; n < 16; ++n)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) row[kPartO + o_col<KV>(n, e, c)] = st.o[n][2 * hh + e] * st.vref;
-    if (c == 0) {
-      row[0] = st.m[hh];
-      row[1] = l[hh];
+    for (int hh = 0; hh < 2; ++hh) {
+      mml[(warp * 16 + g + 8 * hh) * 2 + 0] = st.m[hh];
+      mml[(warp * 16 + g + 8 * hh) * 2 + 1] = l[hh];
     }
   }
+  named_barrier_sync(1, NT);
+  // common max of each of this warp's rows over the warps sharing its head group
+  float f[2];
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    const int r = g + 8 * hh;
+    float M = -INFINITY;
+    for (int w = hg; w < C::kConsumers; w += HG) M = fmaxf(M, mml[(w * 16 + r) * 2]);
+    f[hh] = (st.m[hh] == -INFINITY) ? 0.f : fast_exp2(st.m[hh] - M) * st.vref;
+  }
+  for (int k = 0; k < C::kConsumers / HG; ++k) {
+    if (warp / HG == k) o_to_smem<KV>(mo + hg * 16 * o_stride<KV>(), st.o, f, k == 0);
+    named_barrier_sync(1, NT);
+  }
+  const int first = cta_of_tile(P.seq.tile_begin[b], gridDim.x, P.total_tiles);
+  const int slot = P.seq.item_begin[b] + (blockIdx.x - first);
+  float *part = P.part + (size_t)slot * H * kPartRow;
+  for (int t = threadIdx.x; t < H * kHeadDim / 4; t += NT) {
+    const int h = t / (kHeadDim / 4), d4 = t % (kHeadDim / 4);
+    reinterpret_cast<float4 *>(part + h * kPartRow + kPartO)[d4] =
+        reinterpret_cast<const float4 *>(mo + h * o_stride<KV>())[d4];
+  }
+  if (threadIdx.x < H) {
+    const int h = threadIdx.x, hgh = h >> 4, r = h & 15;
+    float M = -INFINITY, L = 0.f;
+    for (int w = hgh; w < C::kConsumers; w += HG) M = fmaxf(M, mml[(w * 16 + r) * 2]);
+    for (int w = hgh; w < C::kConsumers; w += HG) {
+      const float m = mml[(w * 16 + r) * 2];
+      if (m != -INFINITY) L += fast_exp2(m - M) * mml[(w * 16 + r) * 2 + 1];
+    }
+    part[h * kPartRow + 0] = M;
+    part[h * kPartRow + 1] = L;
+  }
+  named_barrier_sync(1, NT);   // the buffers are clean before any warp's next flush
 }
 
 template <int KV, int HG>
@@ -248,7 +286,7 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, 1)
     const int g = wk.step(P, it);
     const int b = wk.b;
     if (b != cur) {
-      if (cur >= 0) flush_partial<KV, HG>(P, cur, grp * 4 + tg, hg, st);
+      if (cur >= 0) flush_partial<KV, HG>(P, cur, hg, st, sm.merge_o, sm.merge_ml);
       cur = b;
       const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(P.q) + (size_t)b * H * kHeadDim;
       load_q_rows<KV>(qb, hg * 16, qa, P.scale_log2, rowf);
@@ -256,11 +294,12 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, 1)
     }
     if (it % C::kGroups != grp) continue;
     const int s = it % C::kStages;
+    if (*sm.abort_flag) continue;   // after a timeout: keep walking, so every flush barrier is met
     if (!mbar_wait(smem_u32(&sm.full[s]), (it / C::kStages) & 1)) {
       record_status(P.status, kStatusTimeout);
       *sm.abort_flag = 1;
+      continue;
     }
-    if (*sm.abort_flag) return;
     const uint8_t *stg = sm.stages + s * C::kStageBytes;
     const int64_t trow = tile_row0(P, b, g);
     const int64_t row0 = P.seq.start[b], row1 = row0 + P.seq.len[b];
@@ -288,7 +327,7 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
   }
-  if (cur >= 0) flush_partial<KV, HG>(P, cur, grp * 4 + tg, hg, st);
+  if (cur >= 0) flush_partial<KV, HG>(P, cur, hg, st, sm.merge_o, sm.merge_ml);
 }
 
 // ------------------------------------------------------------------ pass 2

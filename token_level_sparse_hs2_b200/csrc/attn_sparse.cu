@@ -8,10 +8,13 @@
 //
 // One CTA per (query row, split of the selected list): every warp gathers its share of each
 // 64-row tile (16-byte cp.async into the swizzled tile layout, two stages) and runs the
-// tensor-core online softmax on 16 heads x 16 rows of it. A row's splits write per-warp
-// partials that merge_partials_kernel combines; a row handled by one CTA is merged in
-// shared memory and written directly.
+// tensor-core online softmax on 16 heads x 16 rows of it. The token groups of a CTA merge in
+// shared memory; the splits of a row form one thread-block cluster and merge through
+// distributed shared memory, each CTA finishing a subset of the heads, so no partial result
+// goes through HBM.
 // merge_partials_kernel (one CTA per output group and head) serves the decode full layer.
+#include <cooperative_groups.h>
+
 #include "attn_pipeline.cuh"
 #include "internal.h"
 
@@ -30,8 +33,10 @@ struct SpCfg {
   static constexpr int kKBytes = (KV == kKvBf16) ? 2 * kBoxBytes : kBoxBytes;
   static constexpr int kStageBytes = (2 * kKBytes + (KV == kKvFp8 ? 512 : 0) + 1023) / 1024 * 1024;
   static constexpr int kStages = 2;
-  // the stage ring doubles as the warp-merge area of a row handled by one CTA
-  static constexpr size_t kMergeBytes = (size_t)kWarps * 16 * (kHeadDim + 2) * 4;
+  // the stage ring doubles as the warp-merge area ([warp][16][128] outputs, [warp][16][2]
+  // max / denominator) followed by the CTA's merged partial ([H][kPartRow]) for the cluster
+  static constexpr size_t kMergeBytes = (size_t)kWarps * 16 * (o_stride<KV>() + 2) * 4 +
+                                        (size_t)16 * HG * kPartRow * 4;
   static constexpr size_t kRegion = ((size_t)kStages * kStageBytes > kMergeBytes)
                                         ? (size_t)kStages * kStageBytes : (kMergeBytes + 1023) / 1024 * 1024;
   static constexpr size_t kSmem = 1024 + kRegion + 2 * kStages * 8 + 16;
@@ -209,34 +214,18 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads) sparse_gather_kernel(
     st.l[h] += __shfl_xor_sync(0xffffffffu, st.l[h], 1);
     st.l[h] += __shfl_xor_sync(0xffffffffu, st.l[h], 2);
   }
-  if (P.n_tsplit > 1) {
-    // this warp's partial: slot ts * TG + tg of row r, its 16 heads (combined by the merge kernel)
-    const int slot = ts * TG + tg;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      float *row = P.part + (((size_t)r * P.n_tsplit * TG + slot) * H + hg * 16 + g + 8 * hh) * kPartRow;
-#pragma unroll
-      for (int n = 0; n < 16; ++n)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) row[kPartO + o_col<KV>(n, e, c)] = st.o[n][2 * hh + e] * st.vref;
-      if (c == 0) {
-        row[0] = st.m[hh];
-        row[1] = st.l[hh];
-      }
-    }
-    return;
-  }
-  // one CTA per row: merge the token groups through shared memory (stages are free once every
-  // warp is past its last tile)
+  // merge the token groups through shared memory (stages are free once every warp is past its
+  // last tile). A CTA that gave up on a wait still takes every barrier below, so that the
+  // cluster's other CTAs never wait for it; its status word already carries the error.
   __syncthreads();
-  if (*abort_flag) return;
-  float *ws_o = reinterpret_cast<float *>(stages);      // [warp][16][128]
-  float *ws_ml = ws_o + C::kWarps * 16 * kHeadDim;      // [warp][16][2]
-#pragma unroll
-  for (int n = 0; n < 16; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      ws_o[(warp * 16 + g + (e >> 1) * 8) * kHeadDim + o_col<KV>(n, e & 1, c)] = st.o[n][e] * st.vref;
+  constexpr int OS = o_stride<KV>();
+  float *ws_o = reinterpret_cast<float *>(stages);      // [warp][16][OS]
+  float *ws_ml = ws_o + C::kWarps * 16 * OS;            // [warp][16][2]
+  float *cpart = ws_ml + C::kWarps * 16 * 2;            // [H][kPartRow]: this CTA's (M, L, O)
+  {
+    const float f[2] = {st.vref, st.vref};
+    o_to_smem<KV>(ws_o + warp * 16 * OS, st.o, f, true);
+  }
   if (c == 0) {
     ws_ml[(warp * 16 + g) * 2 + 0] = st.m[0];
     ws_ml[(warp * 16 + g) * 2 + 1] = st.l[0];
@@ -257,23 +246,76 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads) sparse_gather_kernel(
       const float m = ws_ml[(w * 16 + rh) * 2];
       const float f = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
       L += f * ws_ml[(w * 16 + rh) * 2 + 1];
-      O += f * ws_o[(w * 16 + rh) * kHeadDim + d];
+      O += f * ws_o[(w * 16 + rh) * OS + d];
     }
-    const float val = O / L;
-    const size_t oi = ((size_t)r * H + h) * kHeadDim + d;
-    if (P.out_f32) reinterpret_cast<float *>(P.out)[oi] = val;
-    else reinterpret_cast<__nv_bfloat16 *>(P.out)[oi] = __float2bfloat16_rn(val);
+    if (P.n_tsplit == 1) {
+      const float val = O / L;
+      const size_t oi = ((size_t)r * H + h) * kHeadDim + d;
+      if (P.out_f32) reinterpret_cast<float *>(P.out)[oi] = val;
+      else reinterpret_cast<__nv_bfloat16 *>(P.out)[oi] = __float2bfloat16_rn(val);
+    } else {
+      float *row = cpart + h * kPartRow;
+      row[kPartO + d] = O;
+      if (d == 0) {
+        row[0] = M;
+        row[1] = L;
+      }
+    }
   }
+  if (P.n_tsplit == 1) return;
+  // cluster merge: CTA `ts` of the row finishes heads ts, ts + n_tsplit, ... one warp per head,
+  // reading every CTA's (M, L, O) of that head from its shared memory
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  const int ns = P.n_tsplit;
+  for (int h = ts + ns * warp; h < H; h += ns * C::kWarps) {
+    float mj = -INFINITY, lj = 0.f;
+    if (lane < ns) {
+      const float *rrow = cluster.map_shared_rank(cpart, lane) + h * kPartRow;
+      mj = rrow[0];
+      lj = rrow[1];
+    }
+    float M = mj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float fj = (mj == -INFINITY) ? 0.f : fast_exp2(mj - M);
+    float L = fj * lj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < ns; ++j) {
+      const float f = __shfl_sync(0xffffffffu, fj, j);
+      const float4 o = reinterpret_cast<const float4 *>(cluster.map_shared_rank(cpart, j) + h * kPartRow + kPartO)[lane];
+      O.x += f * o.x;
+      O.y += f * o.y;
+      O.z += f * o.z;
+      O.w += f * o.w;
+    }
+    const float inv = 1.f / L;
+    const size_t oi = ((size_t)r * H + h) * kHeadDim + 4 * lane;
+    if (P.out_f32) {
+      *reinterpret_cast<float4 *>(reinterpret_cast<float *>(P.out) + oi) =
+          make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+    } else {
+      *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(P.out) + oi) =
+          make_uint2(pack_bf16(O.x * inv, O.y * inv), pack_bf16(O.z * inv, O.w * inv));
+    }
+  }
+  cluster.sync();   // no CTA leaves while another may still read its shared memory
 }
 
-// One CTA per (group, head): 8 slot lanes x 32 lanes of 4 output dims; float4 loads.
+// One CTA per (group, head, quarter of head_dim): 32 slot lanes x 8 lanes of 4 output dims,
+// float4 loads, so a group with many slots still spreads over 4 * heads CTAs.
 constexpr int kMergeThreads = 256;
+constexpr int kMergeChunks = 4;
 
 __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __grid_constant__ MergeParams P) {
   __shared__ float red_m[kMergeThreads / 32];
-  __shared__ float red_l[8];
-  __shared__ float4 red_o[8][32];
-  const int grp = blockIdx.x / P.n_heads, h = blockIdx.x % P.n_heads;
+  __shared__ float red_l[32];
+  __shared__ float4 red_o[32][8];
+  const int ch = blockIdx.x % kMergeChunks;
+  const int grp = blockIdx.x / kMergeChunks / P.n_heads, h = blockIdx.x / kMergeChunks % P.n_heads;
   int s0, n;
   if (P.by_seq) {
     s0 = P.seq.item_begin[grp];
@@ -282,51 +324,51 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __g
     s0 = grp * P.n_fixed;
     n = P.n_fixed;
   }
-  if (n <= 1) return;
   griddep_launch_dependents();
   griddep_wait();   // partials come from the previous kernel
   const int H = P.n_heads;
-  const int sl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float m = -INFINITY;
   for (int i = threadIdx.x; i < n; i += kMergeThreads)
     m = fmaxf(m, __ldcg(P.part + ((size_t)(s0 + i) * H + h) * kPartRow));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red_m[sl] = m;
+  if (lane == 0) red_m[w] = m;
   __syncthreads();
   float M = red_m[0];
 #pragma unroll
   for (int i = 1; i < kMergeThreads / 32; ++i) M = fmaxf(M, red_m[i]);
+  const int sl = w * 4 + (lane >> 3), dq = lane & 7;   // slot lane 0..31, dim quad 0..7
   float L = 0.f;
   float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int i = sl; i < n; i += 8) {
+#pragma unroll 2
+  for (int i = sl; i < n; i += 32) {
     const float *row = P.part + ((size_t)(s0 + i) * H + h) * kPartRow;
     const float mi = __ldcg(row);
     const float f = (mi == -INFINITY) ? 0.f : fast_exp2(mi - M);
     L += f * __ldcg(row + 1);
-    const float4 o = __ldcg(reinterpret_cast<const float4 *>(row + kPartO) + lane);
+    const float4 o = __ldcg(reinterpret_cast<const float4 *>(row + kPartO) + ch * 8 + dq);
     O.x += f * o.x;
     O.y += f * o.y;
     O.z += f * o.z;
     O.w += f * o.w;
   }
-  red_o[sl][lane] = O;
-  if (lane == 0) red_l[sl] = L;
+  red_o[sl][dq] = O;
+  if (dq == 0) red_l[sl] = L;
   __syncthreads();
-  if (sl == 0) {
+  if (threadIdx.x < 8) {
     float Lt = 0.f;
     float4 Ot = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
       Lt += red_l[k];
-      Ot.x += red_o[k][lane].x;
-      Ot.y += red_o[k][lane].y;
-      Ot.z += red_o[k][lane].z;
-      Ot.w += red_o[k][lane].w;
+      Ot.x += red_o[k][threadIdx.x].x;
+      Ot.y += red_o[k][threadIdx.x].y;
+      Ot.z += red_o[k][threadIdx.x].z;
+      Ot.w += red_o[k][threadIdx.x].w;
     }
     const float inv = 1.f / Lt;
-    const size_t oi = ((size_t)grp * H + h) * kHeadDim + 4 * lane;
+    const size_t oi = ((size_t)grp * H + h) * kHeadDim + ch * 32 + 4 * threadIdx.x;
     if (P.out_f32) {
       *reinterpret_cast<float4 *>(reinterpret_cast<float *>(P.out) + oi) =
           make_float4(Ot.x * inv, Ot.y * inv, Ot.z * inv, Ot.w * inv);
@@ -335,7 +377,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __g
       *reinterpret_cast<uint2 *>(o) = make_uint2(pack_bf16(Ot.x * inv, Ot.y * inv),
                                                  pack_bf16(Ot.z * inv, Ot.w * inv));
     }
-    if (P.lse && lane == 0) P.lse[(size_t)grp * H + h] = (M + __log2f(Lt)) * kLn2;
+    if (P.lse && ch == 0 && threadIdx.x == 0) P.lse[(size_t)grp * H + h] = (M + __log2f(Lt)) * kLn2;
   }
 }
 
@@ -347,17 +389,60 @@ cudaError_t launch_sparse_t(const SparseParams &p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (e != cudaSuccess) return e;
   const int grid = p.batch * p.n_q * p.n_tsplit;
-  e = launch_pdl(kern, grid, C::kThreads, C::kSmem, s, p);
+  if (p.n_tsplit == 1) {
+    e = launch_pdl(kern, grid, C::kThreads, C::kSmem, s, p);
+  } else {
+    if (p.n_tsplit > 8) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_pdl_cluster(kern, grid, C::kThreads, C::kSmem, p.n_tsplit, s, p);
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// Largest cluster (<= 16) of which at least one can be resident at a time.
+template <int KV, int HG>
+int max_cluster_t() {
+  using C = SpCfg<KV, HG>;
+  auto kern = sparse_gather_kernel<KV, HG>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
+  for (int cs = 16; cs > 1; --cs) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) return cs;
+    cudaGetLastError();
+  }
+  return 1;
 }
 
 }  // namespace
 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t s) {
-  cudaError_t e = launch_pdl(merge_partials_kernel, p.n_groups * p.n_heads, kMergeThreads, 0, s, p);
+  cudaError_t e = launch_pdl(merge_partials_kernel, p.n_groups * p.n_heads * kMergeChunks, kMergeThreads, 0, s, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+int sparse_max_cluster(int kv_dtype, int n_heads) {
+  const int hg = n_heads / 16;
+  if (kv_dtype == HS2_KV_BF16) return hg == 1 ? max_cluster_t<kKvBf16, 1>() : max_cluster_t<kKvBf16, 2>();
+  return hg == 1 ? max_cluster_t<kKvFp8, 1>() : max_cluster_t<kKvFp8, 2>();
 }
 
 cudaError_t launch_sparse(int kv_dtype, const SparseParams &p, cudaStream_t s) {

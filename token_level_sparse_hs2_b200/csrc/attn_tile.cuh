@@ -308,6 +308,51 @@ __device__ __forceinline__ void pv_tile(const uint32_t (&pa)[NT / 2][4], uint32_
   }
 }
 
+// Row stride (floats) of a shared-memory block holding output rows for o_to_smem: with it, the
+// float2 (bf16 layout) or float4 (e4m3 layout) accesses of a warp hit every bank once.
+template <int KV>
+constexpr int o_stride() { return KV == kKvBf16 ? 136 : 144; }
+
+// Stores (first) or adds this warp's output fragments, row hh scaled by f[hh], into rows
+// g and g + 8 of a [16][o_stride<KV>()] float block at base, in head_dim order.
+template <int KV>
+__device__ __forceinline__ void o_to_smem(float *base, const float (&o)[16][4],
+                                          const float (&f)[2], bool first) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    float *row = base + (g + 8 * hh) * o_stride<KV>();
+    if (KV == kKvBf16) {
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        float2 *p = reinterpret_cast<float2 *>(row + n * 8 + 2 * c);
+        float2 v = make_float2(o[n][2 * hh] * f[hh], o[n][2 * hh + 1] * f[hh]);
+        if (!first) {
+          const float2 u = *p;
+          v.x += u.x;
+          v.y += u.y;
+        }
+        *p = v;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 *p = reinterpret_cast<float4 *>(row + 16 * j + 4 * c);
+        float4 v = make_float4(o[2 * j][2 * hh] * f[hh], o[2 * j + 1][2 * hh] * f[hh],
+                               o[2 * j][2 * hh + 1] * f[hh], o[2 * j + 1][2 * hh + 1] * f[hh]);
+        if (!first) {
+          const float4 u = *p;
+          v.x += u.x;
+          v.y += u.y;
+          v.z += u.z;
+          v.w += u.w;
+        }
+        *p = v;
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ online softmax
 
 // State of one warp over its 16 head rows (this lane owns rows g and g+8).

@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -16,6 +17,14 @@
 #include <mutex>
 
 #include "internal.h"
+
+namespace hs2 {
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+unsigned long long launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
+}  // namespace hs2
 
 namespace hs2 {
 
@@ -41,7 +50,7 @@ constexpr int kMaxStreamCtas = 296;       // persistent decode grid, at most
 constexpr int kSegLen = 16384;            // top-k candidates per CTA when rows are split
 constexpr int kManyRows = 148;            // rows at least this many: one CTA per row
 constexpr int kCandCapGlobal = 8192;
-constexpr int kMaxSplit = 32;             // sparse-layer CTAs per query row, at most
+constexpr int kMaxSplit = 16;             // sparse-layer CTAs (one cluster) per query row, at most
 constexpr int kRowsPerBlock = 128;        // (query, head) rows per pass-1 CTA for chunks
 constexpr int kQueriesPass2 = 8;          // queries per pass-2 CTA for chunks
 constexpr size_t kAlign = 256;
@@ -66,8 +75,8 @@ struct Plan {
   bool sparse_split = false;
   // workspace (byte offsets); [0, zero_end) is cleared at the start of every call
   size_t off_status = 0, off_cnt_rows = 0, off_hist = 0, off_cand_count = 0, off_arrive = 0,
-         off_cnt_sp = 0, zero_end = 0;
-  size_t off_part_p1 = 0, off_part_rows = 0, off_cand_key = 0, off_cand_idx = 0, off_part_sp = 0, total = 0;
+         zero_end = 0;
+  size_t off_part_p1 = 0, off_part_rows = 0, off_cand_key = 0, off_cand_idx = 0, total = 0;
 };
 
 hs2_status validate_view(const hs2_kv_view *kv) {
@@ -154,7 +163,6 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   P.off_hist = o; o = align_up(o + (P.n_seg > 1 ? 4 * (size_t)kHistBins * P.n_rows : 0));
   P.off_cand_count = o; o = align_up(o + 4 * (size_t)P.n_rows);
   P.off_arrive = o; o = align_up(o + 4 * (size_t)P.n_rows);
-  P.off_cnt_sp = o; o = align_up(o + 4 * (size_t)P.n_rows * (P.H / 16));
   P.zero_end = o;
   const size_t part_row = (size_t)P.H * kPartRow * 4;
   const size_t max_slots =
@@ -165,8 +173,6 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   const size_t cand = (P.n_seg > 1) ? (size_t)P.n_rows * kCandCapGlobal * 4 : 0;
   P.off_cand_key = o; o = align_up(o + cand);
   P.off_cand_idx = o; o = align_up(o + cand);
-  P.off_part_sp = o;
-  o = align_up(o + (P.sparse_split ? (size_t)P.n_rows * kMaxSplit * 4 * P.H * kPartRow * 4 : 0));
   P.total = o;
 }
 
@@ -301,6 +307,24 @@ NoallocLayout noalloc_layout(const Plan &P) {
 
 bool valid_scale(float s) { return std::isfinite(s) && s > 0.f; }
 
+// largest sparse-layer cluster on the current device (cached per device, cache type, heads)
+hs2_status sparse_cluster_limit(int kv_dtype, int n_heads, int *out) {
+  static std::mutex mu;
+  static int cache[64][2][2] = {};
+  int dev = 0;
+  hs2_status st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != HS2_OK) return st;
+  const int kd = kv_dtype == HS2_KV_BF16 ? 0 : 1, hg = n_heads == 16 ? 0 : 1;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) {
+    *out = 1;
+    return HS2_OK;
+  }
+  if (cache[dev][kd][hg] == 0) cache[dev][kd][hg] = sparse_max_cluster(kv_dtype, n_heads);
+  *out = cache[dev][kd][hg];
+  return HS2_OK;
+}
+
 // multiprocessors of the current device (cached per device)
 hs2_status sm_count(int *out) {
   static std::mutex mu;
@@ -364,6 +388,7 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
     hs2_status st = cuda_check(launch_rows_pass(0, P.kv_dtype, tm, r1, stream), "chunk pass 1");
     if (st != HS2_OK) return st;
     if (mark && (st = (*mark)()) != HS2_OK) return st;
+    if (mark && (st = (*mark)()) != HS2_OK) return st;  // pass 1 merged its own partials
     st = cuda_check(launch_rows_pass(1, P.kv_dtype, tm, r2, stream), "chunk score pass 2");
     if (st != HS2_OK) return st;
     if (mark && (st = (*mark)()) != HS2_OK) return st;
@@ -406,6 +431,7 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   dp.status = ws_at<uint32_t>(ws, P.off_status);
   st = cuda_check(launch_decode_pass(0, P.kv_dtype, tm, dp, stream), "full-attention pass 1");
   if (st != HS2_OK) return st;
+  if (mark && (st = (*mark)()) != HS2_OK) return st;
   {
     MergeParams mp;
     memset(&mp, 0, sizeof mp);
@@ -485,8 +511,12 @@ hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const
   const int64_t cap = std::min<int64_t>(idx_stride, P.max_p + 1);
   const int tiles = (int)((cap + kTile - 1) / kTile);
   int ts = 1;
-  if (P.sparse_split)   // about one CTA per SM: spread the gather over the chip
-    ts = std::max(1, std::min({(kManyRows + P.n_rows - 1) / P.n_rows, tiles, kMaxSplit}));
+  if (P.sparse_split) {   // about one CTA per SM: spread the gather over the chip
+    int max_cluster = 1;
+    hs2_status st = sparse_cluster_limit(P.kv_dtype, P.H, &max_cluster);
+    if (st != HS2_OK) return st;
+    ts = std::max(1, std::min({(kManyRows + P.n_rows - 1) / P.n_rows, tiles, kMaxSplit, max_cluster}));
+  }
   const int tiles_per = (tiles + ts - 1) / ts;
   sp.split_len = tiles_per * kTile;
   sp.n_tsplit = (int)((cap + sp.split_len - 1) / sp.split_len);
@@ -501,22 +531,8 @@ hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const
   sp.v_scale = kv->v_scale;
   sp.out = out;
   sp.out_f32 = out_f32;
-  sp.part = ws_at<float>(ws, P.off_part_sp);
-  sp.counter = ws_at<int32_t>(ws, P.off_cnt_sp);
   sp.status = ws_at<uint32_t>(ws, P.off_status);
-  hs2_status st = cuda_check(launch_sparse(P.kv_dtype, sp, stream), "sparse gather attention");
-  if (st != HS2_OK || sp.n_tsplit == 1) return st;
-  MergeParams mp;
-  memset(&mp, 0, sizeof mp);
-  mp.by_seq = 0;
-  mp.n_groups = P.n_rows;
-  mp.n_fixed = sp.n_tsplit * 4;   // per-warp partial slots per row: splits x token groups
-  mp.n_heads = P.H;
-  mp.part = sp.part;
-  mp.out = out;
-  mp.out_f32 = out_f32;
-  mp.lse = nullptr;
-  return cuda_check(launch_merge(mp, stream), "sparse merge");
+  return cuda_check(launch_sparse(P.kv_dtype, sp, stream), "sparse gather attention");
 }
 
 hs2_status check_budget(int topk, int window) {
@@ -691,8 +707,8 @@ static hs2_status block_impl(const hs2_kv_view *kv, const void *q_full,
       return fail(HS2_ERR_INVALID_ARG, "sparse layer %d: q / out must be 16-byte aligned", l);
   }
   if (events) {
-    if (n_events != 5 + n_sparse)
-      return fail(HS2_ERR_INVALID_ARG, "n_events %d != 5 + n_sparse", n_events);
+    if (n_events != 6 + n_sparse)
+      return fail(HS2_ERR_INVALID_ARG, "n_events %d != 6 + n_sparse", n_events);
     for (int e = 0; e < n_events; ++e)
       if (!events[e]) return fail(HS2_ERR_INVALID_ARG, "event %d is NULL", e);
   }
@@ -780,5 +796,7 @@ const char *hs2_status_string(hs2_status s) {
 }
 
 int32_t hs2_version(void) { return HS2_VERSION; }
+
+uint64_t hs2_launch_count(void) { return hs2::launches_so_far(); }
 
 }  // extern "C"

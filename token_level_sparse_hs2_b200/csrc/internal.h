@@ -19,7 +19,7 @@ constexpr int kHistBins = 2048;
 constexpr int kPartRow = 4 + 128;
 constexpr int kPartO = 4;       // top radix digit: bits [31:21] of the fp32 score
 // decode pass 1: partial slots per (CTA, sequence) -- one per token group of consumer warps
-constexpr int decode_slots_per_cta(int n_heads) { return n_heads == 16 ? 8 : 4; }
+constexpr int decode_slots_per_cta(int) { return 1; }   // warps merge in shared memory first
 
 // device status bits (written into the workspace, read by hs2_read_device_status)
 constexpr uint32_t kStatusTimeout = 1u;
@@ -88,7 +88,7 @@ struct RowsParams {
 struct SparseParams {
   SeqTable seq;
   int32_t batch, n_q, n_heads;
-  int32_t n_tsplit;         // CTAs per row along the selected list
+  int32_t n_tsplit;         // CTAs per row along the selected list (one thread-block cluster)
   int32_t split_len;        // selected entries per CTA (multiple of 64)
   float scale_log2;
   const void *q;            // bf16 [B, n_q, H, 128]
@@ -99,10 +99,11 @@ struct SparseParams {
   const float *k_scale, *v_scale;
   void *out;
   int32_t out_f32;
-  float *part;              // [B*n_q, n_tsplit * 4, H, kPartRow] per-warp partials (n_tsplit > 1)
-  int32_t *counter;         // unused
   uint32_t *status;
 };
+
+// Largest thread-block cluster the sparse layer may use for this cache type and head count.
+int sparse_max_cluster(int kv_dtype, int n_heads);
 
 // Top-k + window selection: n_seg CTAs per query row, each over seg_len candidate positions.
 struct TopkParams {
@@ -150,5 +151,9 @@ cudaError_t launch_rows_pass(int pass, int kv_dtype, const TensorMaps &tm, const
 cudaError_t launch_sparse(int kv_dtype, const SparseParams &p, cudaStream_t s);
 cudaError_t launch_topk(const TopkParams &p, int n_rows, cudaStream_t s);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t s);
+
+// Counts one successful kernel launch (every launch of the library goes through launch_pdl).
+void note_launch();
+unsigned long long launches_so_far();
 
 }  // namespace hs2
