@@ -133,7 +133,8 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   P.tile_begin[P.B] = P.total_tiles;
   // multi-token chunks
   if (P.n_q > 1) {
-    const int qpb1 = kRowsPerBlock / P.H, qpb2 = kQueriesPass2;
+    const int qpb1 = kRowsPerBlock / P.H;
+    const int qpb2 = (P.kv_dtype == HS2_KV_BF16) ? rows_score_tc_queries(P.H) : kQueriesPass2;
     P.n_blk1 = P.n_blk2 = 0;
     for (int b = 0; b < P.B; ++b) {
       P.blk1_begin[b] = P.n_blk1;
@@ -382,14 +383,16 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
     r1.q_per_block = kRowsPerBlock / P.H;
     r1.n_chunks = P.n_chunks1;
     r1.n_items = P.n_blk1 * P.n_chunks1;
-    r2.q_per_block = kQueriesPass2;
+    r2.q_per_block = (P.kv_dtype == HS2_KV_BF16) ? rows_score_tc_queries(P.H) : kQueriesPass2;
     r2.n_chunks = P.n_chunks2;
     r2.n_items = P.n_blk2 * P.n_chunks2;
     hs2_status st = cuda_check(launch_rows_pass(0, P.kv_dtype, tm, r1, stream), "chunk pass 1");
     if (st != HS2_OK) return st;
     if (mark && (st = (*mark)()) != HS2_OK) return st;
     if (mark && (st = (*mark)()) != HS2_OK) return st;  // pass 1 merged its own partials
-    st = cuda_check(launch_rows_pass(1, P.kv_dtype, tm, r2, stream), "chunk score pass 2");
+    st = cuda_check(P.kv_dtype == HS2_KV_BF16 ? launch_rows_score_tc(tm, r2, stream)
+                                              : launch_rows_pass(1, P.kv_dtype, tm, r2, stream),
+                    "chunk score pass 2");
     if (st != HS2_OK) return st;
     if (mark && (st = (*mark)()) != HS2_OK) return st;
     return HS2_OK;

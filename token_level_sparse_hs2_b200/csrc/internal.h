@@ -151,6 +151,10 @@ cudaError_t launch_rows_pass(int pass, int kv_dtype, const TensorMaps &tm, const
 cudaError_t launch_sparse(int kv_dtype, const SparseParams &p, cudaStream_t s);
 cudaError_t launch_topk(const TopkParams &p, int n_rows, cudaStream_t s);
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t s);
+// Score pass 2 of a bf16 cache for n_q > 1 on tcgen05 (blocks of rows_score_tc_queries(H)
+// queries).
+cudaError_t launch_rows_score_tc(const TensorMaps &tm, const RowsParams &p, cudaStream_t s);
+int rows_score_tc_queries(int n_heads);
 
 // Counts one successful kernel launch (every launch of the library goes through launch_pdl).
 void note_launch();
