@@ -54,12 +54,30 @@ def parse():
 
 
 def peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]),
+                "measured")
     except Exception:
-        return 6650.0, "fallback"
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def causal_pairs(w) -> int:
+    """Sum over query rows of the visible prefix length p + 1."""
+    tot = 0
+    for t in w.kv_len.astype(np.int64):
+        first = int(t) - w.n_q + 1
+        tot += w.n_q * first + w.n_q * (w.n_q - 1) // 2
+    return tot
+
+
+def tensor_flops(w) -> dict:
+    """Dense FLOPs of the full layer: per visible (query, token) pair and head, 2 * 128 for
+    q.k and 2 * 128 for p.v (pass 1), 2 * 128 for q.k again (score pass)."""
+    pairs = causal_pairs(w) * w.n_heads
+    return dict(pass1=pairs * 4 * w.head_dim, pass2=pairs * 2 * w.head_dim)
 
 
 def algorithmic_bytes(w) -> dict:
@@ -323,7 +341,7 @@ def main():
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": float(ems.item())}
 
-    hbm, how = peaks()
+    hbm, tf_burst, tf_sust, how = peaks()
     ab = algorithmic_bytes(w)
     p1_s = per["pass1"] / 1e3
     ach = ab["pass1"] / p1_s / 1e9
@@ -333,6 +351,25 @@ def main():
             traffic = json.load(f).get(w.name, {}).get("pass1")
     except Exception:
         pass
+    if w.n_q == 1:   # decode: the passes stream the cache once each (HBM-bound)
+        roofline = {"kernel": "full-attention pass 1", "bound": "hbm", "achieved": ach,
+                    "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": traffic,
+                    "peak_source": how + " copy bandwidth", "bytes_per_launch": ab["pass1"],
+                    "ms_per_launch": per["pass1"]}
+        extra = {}
+    else:            # chunks / prefill: dense products over the causal prefix (tensor-bound)
+        fl = tensor_flops(w)
+        a1 = fl["pass1"] / p1_s / 1e12
+        a2 = fl["pass2"] / (per["pass2"] / 1e3) / 1e12
+        roofline = {"kernel": "full-attention pass 1", "bound": "tensor", "achieved": a1,
+                    "peak": tf_sust, "unit": "TFLOP/s", "frac": a1 / tf_sust, "traffic": traffic,
+                    "peak_source": how + " bf16 GEMM, sustained (kernel inside a long step)",
+                    "flops_per_launch": fl["pass1"], "ms_per_launch": per["pass1"]}
+        extra = {"score_pass_roofline": {
+            "kernel": "score pass 2 (tcgen05)" if w.kv_dtype == "bf16" else "score pass 2",
+            "bound": "tensor", "achieved": a2, "peak": tf_sust, "unit": "TFLOP/s",
+            "frac": a2 / tf_sust, "frac_of_burst_peak": a2 / tf_burst,
+            "flops_per_launch": fl["pass2"], "ms_per_launch": per["pass2"]}}
     line = {
         "metric": METRIC, "value": world * R / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,
@@ -342,10 +379,8 @@ def main():
         "config": dict(config_of(w), parallelism=f"replicas x{world} (independent batches)",
                        l2="inputs larger than L2 (K/V cache %.0f MB > 126 MB); no flush"
                           % (w.k.nbytes * 2 / 1e6)),
-        "roofline": {"kernel": "full-attention pass 1", "bound": "hbm", "achieved": ach,
-                     "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": traffic,
-                     "peak_source": how, "bytes_per_launch": ab["pass1"],
-                     "ms_per_launch": per["pass1"]},
+        "roofline": roofline,
+        **extra,
         "block_roofline": {"bytes_per_step": ab["total"],
                            "achieved_gbs": ab["total"] / (ms_max / 1e3) / 1e9,
                            "frac": ab["total"] / (ms_max / 1e3) / 1e9 / hbm},

@@ -8,16 +8,20 @@
 // s[t] = sum_h exp(c q_h . k_t - lse_h), with lse_h from the output pass.
 //
 // One CTA per (block of 256 / H queries, chunk of the block's causal prefix). For every
-// 128-row K tile the product D = K_tile . Q_block^T (M = 128 tokens, N = 256 (query, head)
-// columns, K = 128) is one chain of 8 tcgen05.mma into a TMEM accumulator. Two accumulators
-// alternate, so the tensor cores fill one while the epilogue drains the other:
-//   warp 9      TMA producer: K tiles (two 64-row halves x two 64-dim boxes) into 4 stages;
+// 128-row K tile the product D = K_tile . Q_block^T - lse / (c log2 e) (M = 128 tokens,
+// N = 256 (query, head) columns) is one chain of 9 tcgen05.mma into a TMEM accumulator: 8
+// steps over head_dim, and a ninth whose A operand is a constant block with ones in its first
+// three columns and whose B operand holds -lse_h log2 e / (c log2 e) of every column split
+// into three bf16 terms (24 significant bits), so the accumulator already carries the
+// log-sum-exp. Two accumulators alternate, so the tensor cores fill one while the epilogue
+// drains the other:
+//   warp 9      TMA producer: K tiles (two 64-row halves x two 64-dim boxes) into 3 stages;
 //   warp 8      MMA issuer (one thread) and TMEM owner (512 columns);
 //   warps 0..7  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (one token each) and
-//               columns 128 (w / 4) .. + 127, computes exp2(c log2e D - lse_h log2e) per
-//               column, sums the H columns of each query and stores s for tokens t <= p.
-// The exponentials (one per token, query and head) bound this pass; the tensor cores run a
-// fraction of their peak beside them.
+//               columns 128 (w / 4) .. + 127, computes exp2(c log2e D) per column, sums the
+//               H columns of each query and stores s for tokens t <= p.
+// The exponentials (one per token, query and head) bound this pass. The special-function
+// unit does most of them; kPolyCols of every 32 go to the FMA pipe instead (exp2_poly2).
 #include "attn_pipeline.cuh"
 #include "internal.h"
 #include "tc05.cuh"
@@ -28,7 +32,8 @@ namespace {
 
 constexpr int kTcTile = 128;                  // cache rows per tile (the MMA's M)
 constexpr int kTcN = 256;                     // (query, head) columns per block (the MMA's N)
-constexpr int kTcStages = 4;
+constexpr int kTcStages = 3;
+constexpr int kPolyCols = 12;                 // of every 32 columns, exponentiated by exp2_poly2
 constexpr int kTcStageBytes = kTcTile * 256;  // two [128][128 B] swizzled dim blocks
 constexpr int kTcEpiWarps = 8;
 constexpr int kTcWarpMma = 8, kTcWarpTma = 9;
@@ -37,18 +42,19 @@ constexpr uint32_t kTcCols = 2 * kTcN;        // two accumulators
 
 struct TcSmem {
   uint8_t *stages, *q;        // stages: kTcStages x 32 KB; q: two [256][128 B] dim blocks
-  float *lse2;                // [256] lse_h log2 e of each column
+  uint8_t *qx, *ones;         // ninth k-step: B [256][128 B] lse terms, A [128][128 B] ones
   uint64_t *full, *empty, *acc_full, *acc_empty, *done;
   uint32_t *tmem_base;
   volatile int *abort_flag;
-  static constexpr size_t kBytes = 1024 + kTcStages * kTcStageBytes + 2 * kTcN * 128 + kTcN * 4 +
-                                   (2 * kTcStages + 5) * 8 + 16;
+  static constexpr size_t kBytes = 1024 + kTcStages * kTcStageBytes + 3 * kTcN * 128 +
+                                   kTcTile * 128 + (2 * kTcStages + 5) * 8 + 16;
   __device__ explicit TcSmem(uint8_t *raw) {
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     stages = base;
     q = stages + kTcStages * kTcStageBytes;
-    lse2 = reinterpret_cast<float *>(q + 2 * kTcN * 128);
-    full = reinterpret_cast<uint64_t *>(lse2 + kTcN);
+    qx = q + 2 * kTcN * 128;
+    ones = qx + kTcN * 128;
+    full = reinterpret_cast<uint64_t *>(ones + kTcTile * 128);
     empty = full + kTcStages;
     acc_full = empty + kTcStages;
     acc_empty = acc_full + 2;
@@ -86,6 +92,51 @@ __device__ __forceinline__ TcGeom tc_geom(const RowsParams &P, int item) {
   g.tile_begin = tile0 + j * ch;
   g.n_tiles = max(0, min(ch, ntl - j * ch));
   return g;
+}
+
+// 2^x for x <= 0 on the FMA pipe (Cody-Waite split x = j + f, j = rint(x) by the 1.5 * 2^23
+// rounding trick, |f| <= 1/2): 2^f from a cubic fitted to minimise the relative error on
+// [-1/2, 1/2] (max 7.5e-5), then j is added to the exponent field. x is clamped at -125 so
+// the exponent cannot wrap; 2^-125 is far below any score's resolution.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = fadd2(x, make_float2(kMagic, kMagic));
+  const float2 r = fadd2(t, make_float2(-kMagic, -kMagic));
+  const float2 f = ffma2(r, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(f, make_float2(0.0551716648f, 0.0551716648f), make_float2(0.2426111251f, 0.2426111251f));
+  p = ffma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
+  p = ffma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// hs[0] / hs[1] = sum of exp2(scale * v[i]) over i < 16 / i >= 16; the first kPolyCols / 2 of
+// each half on the FMA pipe, the rest on the special-function unit.
+__device__ __forceinline__ void exp2_sum16x2(const float (&v)[32], float scale, float (&hs)[2]) {
+  const float2 sc = make_float2(scale, scale);
+  float2 e[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int half = k >> 3, kk = k & 7;   // pair kk of half `half`: columns 16 half + 2 kk
+    const float2 x = ffma2(make_float2(v[16 * half + 2 * kk], v[16 * half + 2 * kk + 1]), sc,
+                           make_float2(0.f, 0.f));
+    if (2 * kk < kPolyCols / 2) {
+      e[k] = exp2_poly2(x);
+    } else {
+      e[k] = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float2 s4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s4[k] = fadd2(e[8 * h + 2 * k], e[8 * h + 2 * k + 1]);
+    const float2 s2a = fadd2(s4[0], s4[1]), s2b = fadd2(s4[2], s4[3]);
+    const float2 s1 = fadd2(s2a, s2b);
+    hs[h] = s1.x + s1.y;
+  }
 }
 
 __device__ __forceinline__ void fail_timeout(const RowsParams &P, volatile int *abort_flag) {
@@ -134,10 +185,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (r < nrows) v = *reinterpret_cast<const uint4 *>(qg + (size_t)r * kHeadDim + ch * 8);
       *reinterpret_cast<uint4 *>(sm.q + (ch >> 3) * (kTcN * 128) + sw128(r, (ch & 7) * 16)) = v;
     }
+    // ninth k-step operands: all 16-byte chunks zero, then the three terms of each row
+    for (int t = threadIdx.x; t < (kTcN + kTcTile) * 8; t += kTcEpiWarps * 32)
+      reinterpret_cast<uint4 *>(sm.qx)[t] = make_uint4(0, 0, 0, 0);   // qx and ones are adjacent
+    named_barrier_sync(1, kTcEpiWarps * 32);
     for (int r = threadIdx.x; r < kTcN; r += kTcEpiWarps * 32) {
-      float l = 0.f;
-      if (r < nrows) l = P.lse[((size_t)G.b * P.n_q + G.i0) * H + r] * kLog2e;
-      sm.lse2[r] = l;
+      float v = 0.f;
+      if (r < nrows) v = -P.lse[((size_t)G.b * P.n_q + G.i0) * H + r] * kLog2e / P.scale_log2;
+      const __nv_bfloat16 h1 = __float2bfloat16_rn(v);
+      const float r1 = v - __bfloat162float(h1);
+      const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 h3 = __float2bfloat16_rn(r1 - __bfloat162float(h2));
+      __nv_bfloat16 *row = reinterpret_cast<__nv_bfloat16 *>(sm.qx + sw128(r, 0));
+      row[0] = h1;
+      row[1] = h2;
+      row[2] = h3;
+      if (r < kTcTile) {
+        __nv_bfloat16 *one = reinterpret_cast<__nv_bfloat16 *>(sm.ones + sw128(r, 0));
+        one[0] = one[1] = one[2] = __float2bfloat16_rn(1.f);
+      }
     }
     fence_proxy_async_smem();
   }
@@ -196,6 +262,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           umma_bf16(tmem + a * kTcN, umma_desc_sw128(st + off, 1024), umma_desc_sw128(qs + qoff, 1024),
                     idesc, k > 0);
         }
+        umma_bf16(tmem + a * kTcN, umma_desc_sw128(smem_u32(sm.ones), 1024),
+                  umma_desc_sw128(smem_u32(sm.qx), 1024), idesc, true);
         umma_commit(smem_u32(&sm.empty[s]));
         umma_commit(smem_u32(&sm.acc_full[a]));
       }
@@ -226,25 +294,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok || *sm.abort_flag) break;
       tc_fence_after();
+      // 4 loads of 32 columns, each issued before the previous one is consumed
       float sum[QH];
 #pragma unroll
       for (int j = 0; j < QH; ++j) sum[j] = 0.f;
+      float va[32], vb[32];
+      const uint32_t col0 = lane_addr + a * kTcN + half * 128;
+      tmem_ld32(col0, va);
+      tmem_wait_ld();
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {                // 32 columns per load
-        float v[32];
-        tmem_ld32(lane_addr + a * kTcN + half * 128 + cb * 32, v);
-        tmem_wait_ld();
-        const float4 *l4 = reinterpret_cast<const float4 *>(sm.lse2 + half * 128 + cb * 32);
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 l = l4[c4];
-          const int j = (cb * 32 + c4 * 4) / H;
-          float x0 = fast_exp2(fmaf(v[4 * c4 + 0], P.scale_log2, -l.x));
-          float x1 = fast_exp2(fmaf(v[4 * c4 + 1], P.scale_log2, -l.y));
-          float x2 = fast_exp2(fmaf(v[4 * c4 + 2], P.scale_log2, -l.z));
-          float x3 = fast_exp2(fmaf(v[4 * c4 + 3], P.scale_log2, -l.w));
-          sum[j] += (x0 + x1) + (x2 + x3);
+      for (int cb = 0; cb < 4; ++cb) {
+        if (cb < 3) {
+          if (cb & 1) tmem_ld32(col0 + (cb + 1) * 32, va);
+          else tmem_ld32(col0 + (cb + 1) * 32, vb);
         }
+        const float (&v)[32] = (cb & 1) ? vb : va;
+        float hs[2];
+        exp2_sum16x2(v, P.scale_log2, hs);
+        const int c0 = cb * 32;
+        if (H == 32) {
+          sum[c0 / 32] += hs[0] + hs[1];
+        } else {
+          sum[c0 / 16] += hs[0];
+          sum[c0 / 16 + 1] += hs[1];
+        }
+        if (cb < 3) tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
