@@ -266,6 +266,24 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+// 2^x for x <= 0 on the FMA pipe (Cody-Waite split x = j + f, j = rint(x) by the 1.5 * 2^23
+// rounding trick, |f| <= 1/2): 2^f from a cubic fitted to minimise the relative error on
+// [-1/2, 1/2] (max 7.5e-5), then j is added to the exponent field. x is clamped at -125 so
+// the exponent cannot wrap; 2^-125 is far below any score's resolution.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = fadd2(x, make_float2(kMagic, kMagic));
+  const float2 r = fadd2(t, make_float2(-kMagic, -kMagic));
+  const float2 f = ffma2(r, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(f, make_float2(0.0551716648f, 0.0551716648f), make_float2(0.2426111251f, 0.2426111251f));
+  p = ffma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
+  p = ffma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // ------------------------------------------------------------------ O += P . V
 
 template <int KV, int NT, int LAYOUT = kSwz>

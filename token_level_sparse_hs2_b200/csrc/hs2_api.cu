@@ -386,7 +386,9 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
     r2.q_per_block = (P.kv_dtype == HS2_KV_BF16) ? rows_score_tc_queries(P.H) : kQueriesPass2;
     r2.n_chunks = P.n_chunks2;
     r2.n_items = P.n_blk2 * P.n_chunks2;
-    hs2_status st = cuda_check(launch_rows_pass(0, P.kv_dtype, tm, r1, stream), "chunk pass 1");
+    hs2_status st = cuda_check(P.kv_dtype == HS2_KV_BF16 ? launch_rows_attn_tc(tm, r1, stream)
+                                                         : launch_rows_pass(0, P.kv_dtype, tm, r1, stream),
+                               "chunk pass 1");
     if (st != HS2_OK) return st;
     if (mark && (st = (*mark)()) != HS2_OK) return st;
     if (mark && (st = (*mark)()) != HS2_OK) return st;  // pass 1 merged its own partials

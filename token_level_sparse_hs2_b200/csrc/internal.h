@@ -155,6 +155,9 @@ cudaError_t launch_merge(const MergeParams &p, cudaStream_t s);
 // queries).
 cudaError_t launch_rows_score_tc(const TensorMaps &tm, const RowsParams &p, cudaStream_t s);
 int rows_score_tc_queries(int n_heads);
+// Output pass 1 of a bf16 cache for n_q > 1 on tcgen05 (blocks of 128 / H queries, the chunk
+// partials and counters of RowsParams).
+cudaError_t launch_rows_attn_tc(const TensorMaps &tm, const RowsParams &p, cudaStream_t s);
 
 // Counts one successful kernel launch (every launch of the library goes through launch_pdl).
 void note_launch();
