@@ -46,6 +46,9 @@ constexpr int kPreTiles = 24;   // tiles whose indices are fetched up front
 
 // This warp's share of tile `it`: rows [w * RPW, (w+1) * RPW), cp.async into stage `st`, then
 // one arrival per lane on `bar` once the copies land (entries past the list are zero-filled).
+// Lane l owns one 16-byte column of the rows (bf16: chunk l % 16 of K (l < 16) or V; e4m3: chunk
+// l % 8 of K or V of every other row), so a copy costs a shuffle of the row's position, one
+// address multiply-add and the swizzled destination. Lanes < RPW hold the rows' positions.
 template <int KV, int HG>
 __device__ __forceinline__ void gather_rows(const SparseParams &P, int64_t seq_row0, int64_t p,
                                             int e_first, int cnt, int warp, uint8_t *st,
@@ -53,42 +56,43 @@ __device__ __forceinline__ void gather_rows(const SparseParams &P, int64_t seq_r
   using C = SpCfg<KV, HG>;
   const int lane = threadIdx.x & 31;
   constexpr int RPW = C::kRowsPerWarp;
-  constexpr int CH = (KV == kKvBf16) ? 16 : 8;        // 16-byte chunks per row
-  constexpr int PER = RPW * CH * 2 / 32;               // copies per lane (K and V)
-#pragma unroll
-  for (int k = 0; k < PER; ++k) {
-    const int q = k * 32 + lane;                       // (row, chunk, K/V) flattened
-    const int kv = q / (RPW * CH);
-    const int rem = q % (RPW * CH);
-    const int rl = rem / CH, ch = rem % CH;
-    const int rr = warp * RPW + rl;
-    const int e = e_first + rr;
-    const bool v = e < cnt;
-    int64_t pos = __shfl_sync(0xffffffffu, pos_lane, rl);
-    if (!v) pos = 0;
-    if (pos < 0 || pos > p) {
+  int32_t mypos = -1;   // validated position of this lane's row, -1 past the list
+  if (lane < RPW && e_first + warp * RPW + lane < cnt) {
+    mypos = pos_lane;
+    if (pos_lane < 0 || pos_lane > p) {
       bad = true;
-      pos = 0;
-    }
-    const int64_t row = seq_row0 + pos;
-    const uint32_t nb = v ? 16u : 0u;
-    if (KV == kKvBf16) {
-      const uint8_t *src = reinterpret_cast<const uint8_t *>(kv ? P.v : P.k) + row * 256 + ch * 16;
-      cp_async_16(smem_u32(st + kv * C::kKBytes + tile_off(kTile, rr, ch * 8)), src, nb);
-    } else {
-      const uint8_t *src = reinterpret_cast<const uint8_t *>(kv ? P.v : P.k) + row * 128 + ch * 16;
-      cp_async_16(smem_u32(st + kv * C::kKBytes + fp8_off(rr, ch * 16)), src, nb);
+      mypos = 0;
     }
   }
-  if (KV == kKvFp8 && lane < RPW) {
-    const int rr = warp * RPW + lane;
-    const bool v = e_first + rr < cnt;
-    int64_t pos = v ? pos_lane : 0;
-    if (pos < 0 || pos > p) pos = 0;
-    const int64_t row = seq_row0 + pos;
-    uint8_t *sc = st + 2 * C::kKBytes;
-    cp_async_4(smem_u32(sc + rr * 4), P.k_scale + row, v ? 4u : 0u);
-    cp_async_4(smem_u32(sc + (kTile + rr) * 4), P.v_scale + row, v ? 4u : 0u);
+  if (KV == kKvBf16) {
+    const int kv = lane >> 4, ch = lane & 15;
+    const uint8_t *src0 = reinterpret_cast<const uint8_t *>(kv ? P.v : P.k) + seq_row0 * 256 + ch * 16;
+    uint8_t *dst0 = st + kv * C::kKBytes + (ch >> 3) * (kTile * 128);
+#pragma unroll
+    for (int rl = 0; rl < RPW; ++rl) {
+      const int rr = warp * RPW + rl;
+      const int32_t pos = __shfl_sync(0xffffffffu, mypos, rl);
+      cp_async_16(smem_u32(dst0 + rr * 128 + (((ch & 7) ^ (rr & 7)) << 4)),
+                  src0 + (int64_t)max(pos, 0) * 256, pos >= 0 ? 16u : 0u);
+    }
+  } else {
+    const int sub = lane >> 4, kv = (lane >> 3) & 1, ch = lane & 7;
+    const uint8_t *src0 = reinterpret_cast<const uint8_t *>(kv ? P.v : P.k) + seq_row0 * 128 + ch * 16;
+    uint8_t *dst0 = st + kv * C::kKBytes;
+#pragma unroll
+    for (int rl = 0; rl < RPW; rl += 2) {
+      const int r2 = rl + sub, rr = warp * RPW + r2;
+      const int32_t pos = __shfl_sync(0xffffffffu, mypos, r2);
+      cp_async_16(smem_u32(dst0 + fp8_off(rr, ch * 16)), src0 + (int64_t)max(pos, 0) * 128,
+                  pos >= 0 ? 16u : 0u);
+    }
+    if (lane < RPW) {
+      const int rr = warp * RPW + lane;
+      const int64_t row = seq_row0 + max(mypos, 0);
+      uint8_t *sc = st + 2 * C::kKBytes;
+      cp_async_4(smem_u32(sc + rr * 4), P.k_scale + row, mypos >= 0 ? 4u : 0u);
+      cp_async_4(smem_u32(sc + (kTile + rr) * 4), P.v_scale + row, mypos >= 0 ? 4u : 0u);
+    }
   }
   cp_async_mbar_arrive(bar);
 }
