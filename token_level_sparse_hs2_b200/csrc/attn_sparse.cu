@@ -25,6 +25,8 @@ namespace {
 // One CTA per (query row, split of its selected list), no dedicated producer: the 4 * HG
 // warps each gather 64 / (4 * HG) rows of every tile with 16-byte cp.async (so the copies are
 // issued from all four SM sub-partitions at once) and each computes 16 heads x 16 rows of it.
+constexpr int kPreTiles = 24;   // tiles whose indices are staged in shared memory up front
+
 template <int KV, int HG>
 struct SpCfg {
   static constexpr int kWarps = 4 * HG;
@@ -39,10 +41,8 @@ struct SpCfg {
                                         (size_t)16 * HG * kPartRow * 4;
   static constexpr size_t kRegion = ((size_t)kStages * kStageBytes > kMergeBytes)
                                         ? (size_t)kStages * kStageBytes : (kMergeBytes + 1023) / 1024 * 1024;
-  static constexpr size_t kSmem = 1024 + kRegion + 2 * kStages * 8 + 16;
+  static constexpr size_t kSmem = 1024 + kRegion + 2 * kStages * 8 + 16 + kPreTiles * kTile * 4;
 };
-
-constexpr int kPreTiles = 24;   // tiles whose indices are fetched up front
 
 // This warp's share of tile `it`: rows [w * RPW, (w+1) * RPW), cp.async into stage `st`, then
 // one arrival per lane on `bar` once the copies land (entries past the list are zero-filled).
@@ -98,7 +98,7 @@ __device__ __forceinline__ void gather_rows(const SparseParams &P, int64_t seq_r
 }
 
 template <int KV, int HG>
-__global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads) sparse_gather_kernel(const __grid_constant__ SparseParams P) {
+__global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kernel(const __grid_constant__ SparseParams P) {
   using C = SpCfg<KV, HG>;
   constexpr int H = 16 * HG;
   constexpr int TG = 4;   // token groups: warp w covers rows [16 * (w / HG), +16) of a tile
@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads) sparse_gather_kernel(
   uint64_t *full = reinterpret_cast<uint64_t *>(stages + C::kRegion);
   uint64_t *empty = full + C::kStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + C::kStages);
+  int32_t *s_idx = const_cast<int32_t *>(reinterpret_cast<volatile int32_t *>(abort_flag + 4));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x / P.n_tsplit, ts = blockIdx.x % P.n_tsplit;
   const int b = r / P.n_q, i = r % P.n_q;
@@ -124,30 +125,21 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads) sparse_gather_kernel(
   griddep_launch_dependents();
   griddep_wait();   // idx / count come from the selection kernel
   const int e_begin = ts * P.split_len;
-  // this warp's row indices for its first kPreTiles tiles, fetched together with the count
+  // the split's first kPreTiles tiles of row indices, staged in shared memory (coalesced)
   const int32_t *idx = P.idx + (size_t)r * P.idx_stride;
-  int32_t pre[kPreTiles];
-#pragma unroll
-  for (int k = 0; k < kPreTiles; ++k) {
-    const int e = e_begin + k * kTile + warp * C::kRowsPerWarp + lane;
-    pre[k] = (lane < C::kRowsPerWarp && k * kTile < P.split_len && e < P.idx_stride) ? __ldcg(idx + e) : 0;
-  }
+  const int n_pre = min(min(P.split_len, kPreTiles * kTile), P.idx_stride - e_begin);
+  for (int t = threadIdx.x; t < n_pre; t += C::kThreads) s_idx[t] = __ldcg(idx + e_begin + t);
   int cnt = __ldcg(P.count + r);
   if (cnt < 1 || cnt > P.idx_stride) {
     if (threadIdx.x == 0) record_status(P.status, kStatusCheck);
     cnt = max(1, min(cnt, P.idx_stride));
   }
   const int n_tiles = max(0, min(P.split_len, cnt - e_begin) + kTile - 1) / kTile;
+  __syncthreads();   // s_idx
   auto pos_of = [&](int it) -> int32_t {
-    int32_t v = 0;
-#pragma unroll
-    for (int k = 0; k < kPreTiles; ++k)
-      if (k == it) v = pre[k];
-    if (it >= kPreTiles) {
-      const int e = e_begin + it * kTile + warp * C::kRowsPerWarp + lane;
-      v = (lane < C::kRowsPerWarp && e < cnt) ? __ldcg(idx + e) : 0;
-    }
-    return v;
+    const int k = it * kTile + warp * C::kRowsPerWarp + lane;   // entry within the split
+    if (lane >= C::kRowsPerWarp || e_begin + k >= cnt) return 0;
+    return (k < n_pre) ? s_idx[k] : __ldcg(idx + e_begin + k);
   };
   bool bad = false;
   for (int it = 0; it < min(n_tiles, C::kStages); ++it)
