@@ -8,9 +8,11 @@
 //
 // One CTA per (block, chunk of the block's causal prefix); per 128-row K/V tile i:
 //   S_i = Q . K_i^T      tcgen05.mma, A = Q block (smem), B = K tile (smem), D = S buffer i % 2
-//   P_i = exp2(c log2e S_i - m)   four softmax warps, one (query, head) row per thread: the
-//                        row max, a lazy rescale, the exponentials (special-function unit and
-//                        exp2_poly2), the row sum; P is written back over S as bf16 pairs
+//   P_i = exp2(c log2e S_i - m)   eight softmax warps, two threads per (query, head) row (warps
+//                        w and w + 4 read the same TMEM lanes, one half of the columns each):
+//                        the row max (halves exchanged through shared memory), a lazy
+//                        rescale, the exponentials (special-function unit and exp2_poly2), the
+//                        row sum; P is written back over S as bf16 pairs
 //   O += P_i . V_i       tcgen05.mma, A = P (TMEM), B = V tile (smem, MN-major), D = O
 // The MMA warp issues S_{i+1} before O += P_i V_i, so the tensor cores compute the next scores
 // while the softmax warps work. The reference max m only moves when a tile's row max exceeds
@@ -28,9 +30,9 @@ constexpr int kA1Tile = 128;                    // cache rows per tile
 constexpr int kA1Rows = 128;                    // (query, head) rows per block
 constexpr int kA1KStages = 3, kA1VStages = 2;
 constexpr int kA1TileBytes = kA1Tile * 256;     // two [128][128 B] swizzled dim blocks
-constexpr int kA1SmWarps = 4;
-constexpr int kA1WarpMma = 4, kA1WarpTma = 5;
-constexpr int kA1Threads = 6 * 32;
+constexpr int kA1SmWarps = 8;
+constexpr int kA1WarpMma = 8, kA1WarpTma = 9;
+constexpr int kA1Threads = 10 * 32;
 constexpr uint32_t kA1Cols = 512;               // S/P buffers at 0 and 128, O at 256
 constexpr uint32_t kA1ColO = 256;
 constexpr float kA1Lazy = 8.f;
@@ -38,18 +40,20 @@ constexpr int kA1PolyPairs = 6;                 // of every 16 pairs, exponentia
 
 struct A1Smem {
   uint8_t *q, *k, *v;
-  uint64_t *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done, *done;
+  float *xm;                  // [2 buffers][2 halves][128 rows] partial row maxima / sums
+  uint64_t *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done, *done, *x_full;
   uint32_t *tmem_base;
   volatile int *abort_flag;
   static constexpr size_t kBytes = 1024 + (size_t)kA1Rows * 256 +
-                                   (size_t)(kA1KStages + kA1VStages) * kA1TileBytes +
-                                   (2 * kA1KStages + 2 * kA1VStages + 6) * 8 + 16;
+                                   (size_t)(kA1KStages + kA1VStages) * kA1TileBytes + 4 * kA1Rows * 4 +
+                                   (2 * kA1KStages + 2 * kA1VStages + 8) * 8 + 16;
   __device__ explicit A1Smem(uint8_t *raw) {
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     q = base;
     k = q + kA1Rows * 256;
     v = k + kA1KStages * kA1TileBytes;
-    k_full = reinterpret_cast<uint64_t *>(v + kA1VStages * kA1TileBytes);
+    xm = reinterpret_cast<float *>(v + kA1VStages * kA1TileBytes);
+    k_full = reinterpret_cast<uint64_t *>(xm + 4 * kA1Rows);
     k_empty = k_full + kA1KStages;
     v_full = k_empty + kA1KStages;
     v_empty = v_full + kA1VStages;
@@ -57,7 +61,8 @@ struct A1Smem {
     p_full = s_full + 2;
     o_done = p_full + 2;
     done = o_done + 1;
-    tmem_base = reinterpret_cast<uint32_t *>(done + 1);
+    x_full = done + 1;
+    tmem_base = reinterpret_cast<uint32_t *>(x_full + 2);
     abort_flag = reinterpret_cast<volatile int *>(tmem_base + 1);
   }
 };
@@ -132,6 +137,8 @@ __global__ void __launch_bounds__(kA1Threads, 1)
     }
     mbar_init(smem_u32(&sm.o_done[0]), 1);
     mbar_init(smem_u32(&sm.done[0]), 1);
+    mbar_init(smem_u32(&sm.x_full[0]), kA1SmWarps * 32);
+    mbar_init(smem_u32(&sm.x_full[1]), kA1SmWarps * 32);
     *sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -230,75 +237,82 @@ __global__ void __launch_bounds__(kA1Threads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = warp * 32 + lane;                  // TMEM lane = (query, head) row
+    const int r = (warp & 3) * 32 + lane;            // TMEM lane = (query, head) row
+    const int half = warp >> 2;                      // columns [64 half, 64 half + 64)
     const int qi = r / H;
     const int64_t plim = G.pfirst + qi;              // last visible position of this row
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sc = P.scale_log2;
     for (int it = 0; it < n; ++it) {
       const int a = it & 1;
       if (!warp_wait(P, sm.abort_flag, &sm.s_full[a], (it >> 1) & 1)) break;
       tc_fence_after();
-      float x[128];
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
+      float x[64];
+      {
         float v[32];
-        tmem_ld32(lane_addr + a * 128 + cb * 32, v);
+        tmem_ld32(lane_addr + a * 128 + half * 64, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[cb * 32 + i] = v[i] * sc;
-      }
-      const int64_t trow = (int64_t)(G.tile_begin + it) * kA1Tile;   // absolute row of column 0
-      const bool full = trow >= G.row0 && trow + kA1Tile - 1 - G.row0 <= G.pfirst;
-      if (!__all_sync(0xffffffffu, full)) {
-        const int64_t lo = G.row0 - trow, hi = G.row0 + plim - trow;   // valid columns [lo, hi]
+        for (int i = 0; i < 32; ++i) x[i] = v[i];
+        tmem_ld32(lane_addr + a * 128 + half * 64 + 32, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
+        for (int i = 0; i < 32; ++i) x[32 + i] = v[i];
+      }
+      const int64_t tcol = (int64_t)(G.tile_begin + it) * kA1Tile + half * 64;   // row of column 0
+      const bool full = tcol >= G.row0 && tcol + 63 - G.row0 <= G.pfirst;
+      if (!__all_sync(0xffffffffu, full)) {
+        const int64_t lo = G.row0 - tcol, hi = G.row0 + plim - tcol;   // valid columns [lo, hi]
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
           if (i < lo || i > hi) x[i] = -INFINITY;
       }
-      float mt = -INFINITY;
+      // partial max of raw scores (sc > 0), exchanged with the thread holding the other half
+      float mh = fmax3(x[0], x[1], x[2]);
 #pragma unroll
-      for (int i = 0; i < 128; ++i) mt = fmaxf(mt, x[i]);
+      for (int i = 3; i < 63; i += 2) mh = fmax3(mh, x[i], x[i + 1]);
+      mh = fmaxf(mh, x[63]);
+      sm.xm[(a * 2 + half) * kA1Rows + r] = mh;
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cnt(smem_u32(&sm.x_full[a]), 32);
+      if (!warp_wait(P, sm.abort_flag, &sm.x_full[a], (it >> 1) & 1)) break;
+      const float mt = fmaxf(mh, sm.xm[(a * 2 + (half ^ 1)) * kA1Rows + r]) * sc;
       const bool move = mt > m_run + kA1Lazy;
       if (__any_sync(0xffffffffu, move)) {
         const float m_new = move ? mt : m_run;
         const float alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
         l_run *= alpha;
         m_run = m_new;
-        if (it > 0) {   // rescale O once the previous P V product has landed
+        if (it > 0) {   // rescale this half of O once the previous P V product has landed
           if (!warp_wait(P, sm.abort_flag, &sm.o_done[0], (it - 1) & 1)) break;
           tc_fence_after();
 #pragma unroll
-          for (int cb = 0; cb < 4; ++cb) {
+          for (int cb = 0; cb < 2; ++cb) {
             float v[32];
-            tmem_ld32(lane_addr + kA1ColO + cb * 32, v);
+            tmem_ld32(lane_addr + kA1ColO + half * 64 + cb * 32, v);
             tmem_wait_ld();
             uint32_t u[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(v[i] * alpha);
-            tmem_st32(lane_addr + kA1ColO + cb * 32, u);
+            tmem_st32(lane_addr + kA1ColO + half * 64 + cb * 32, u);
           }
           tmem_wait_st();
         }
       }
       const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-      const float2 neg = make_float2(-mref, -mref);
+      const float2 sc2 = make_float2(sc, sc), neg = make_float2(-mref, -mref);
       float2 ls = make_float2(0.f, 0.f);
+      uint32_t pk[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const int i = half * 64 + 2 * k;
-          const float2 z = fadd2(make_float2(x[i], x[i + 1]), neg);
-          float2 e;
-          if ((k & 15) < kA1PolyPairs) e = exp2_poly2(z);
-          else e = make_float2(fast_exp2(z.x), fast_exp2(z.y));
-          ls = fadd2(ls, e);
-          pk[k] = pack_bf16(e.x, e.y);
-        }
-        tmem_st32(lane_addr + a * 128 + half * 32, pk);
+      for (int k = 0; k < 32; ++k) {
+        const float2 z = ffma2(make_float2(x[2 * k], x[2 * k + 1]), sc2, neg);
+        float2 e;
+        if ((k & 15) < kA1PolyPairs) e = exp2_poly2(z);
+        else e = make_float2(fast_exp2(z.x), fast_exp2(z.y));
+        ls = fadd2(ls, e);
+        pk[k] = pack_bf16(e.x, e.y);
       }
+      tmem_st32(lane_addr + a * 128 + half * 32, pk);
       l_run += ls.x + ls.y;
       tmem_wait_st();
       tc_fence_before();
@@ -310,17 +324,21 @@ __global__ void __launch_bounds__(kA1Threads, 1)
   __syncthreads();   // the MMA warp has seen every product land (done barrier)
   tc_fence_after();
   const bool aborted = *sm.abort_flag != 0;
+  if (warp < kA1SmWarps) sm.xm[(warp >> 2) * kA1Rows + (warp & 3) * 32 + lane] = l_run;
+  __syncthreads();
   if (warp < kA1SmWarps && !aborted) {
     // ------------------------------------------------------------ output or chunk partial
-    const int r = warp * 32 + lane;
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int r = (warp & 3) * 32 + lane, half = warp >> 2;
+    const float l_row = sm.xm[r] + sm.xm[kA1Rows + r];
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const size_t orow = ((size_t)G.b * P.n_q + G.i0) * H + r;
     float *part = P.part + (((size_t)G.blk_global * P.n_chunks + G.j) * kA1Rows + r) * kPartRow;
-    const float inv = (P.n_chunks == 1) ? 1.f / l_run : 1.f;
+    const float inv = (P.n_chunks == 1) ? 1.f / l_row : 1.f;
 #pragma unroll
-    for (int cb = 0; cb < 4; ++cb) {
+    for (int cb = 0; cb < 2; ++cb) {
+      const int c0 = half * 64 + cb * 32;
       float v[32];
-      tmem_ld32(lane_addr + kA1ColO + cb * 32, v);
+      tmem_ld32(lane_addr + kA1ColO + c0, v);
       tmem_wait_ld();
       if (n == 0) {
 #pragma unroll
@@ -329,15 +347,15 @@ __global__ void __launch_bounds__(kA1Threads, 1)
       if (P.n_chunks > 1) {
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4 *>(part + kPartO + cb * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          *reinterpret_cast<float4 *>(part + kPartO + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
       } else if (r < nrows) {
         if (P.out_f32) {
-          float *o = reinterpret_cast<float *>(P.out) + orow * kHeadDim + cb * 32;
+          float *o = reinterpret_cast<float *>(P.out) + orow * kHeadDim + c0;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *reinterpret_cast<float4 *>(o + i) = make_float4(v[i] * inv, v[i + 1] * inv, v[i + 2] * inv, v[i + 3] * inv);
         } else {
-          __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(P.out) + orow * kHeadDim + cb * 32;
+          __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(P.out) + orow * kHeadDim + c0;
 #pragma unroll
           for (int i = 0; i < 32; i += 8)
             *reinterpret_cast<uint4 *>(o + i) =
@@ -346,11 +364,13 @@ __global__ void __launch_bounds__(kA1Threads, 1)
         }
       }
     }
-    if (P.n_chunks > 1) {
-      part[0] = m_run;
-      part[1] = l_run;
-    } else if (r < nrows) {
-      P.lse[orow] = (m_run + __log2f(l_run)) * kLn2;
+    if (half == 0) {
+      if (P.n_chunks > 1) {
+        part[0] = m_run;
+        part[1] = l_row;
+      } else if (r < nrows) {
+        P.lse[orow] = (m_run + __log2f(l_row)) * kLn2;
+      }
     }
   }
   tc_fence_before();
