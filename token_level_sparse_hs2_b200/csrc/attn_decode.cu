@@ -98,7 +98,7 @@ __device__ void produce_stream(const TensorMaps &tm, const DecodeParams &P, uint
   using C = StreamCfg<KV, HG, PASS>;
   const int lane = threadIdx.x & 31;
   TileWalk wk(P, PASS == 1);
-  griddep_wait();
+  if (PASS == 0) griddep_wait();   // pass 2 streams K, which no earlier kernel writes
   for (int it = 0; it < wk.n; ++it) {
     const int g = wk.step(P, it);
     const int s = it % C::kStages;

@@ -38,7 +38,7 @@ struct SpCfg {
   // the stage ring doubles as the warp-merge area ([warp][16][128] outputs, [warp][16][2]
   // max / denominator) followed by the CTA's merged partial ([H][kPartRow]) for the cluster
   static constexpr size_t kMergeBytes = (size_t)kWarps * 16 * (o_stride<KV>() + 2) * 4 +
-                                        (size_t)16 * HG * kPartRow * 4;
+                                        (size_t)16 * HG * (kPartRow + 2) * 4;
   static constexpr size_t kRegion = ((size_t)kStages * kStageBytes > kMergeBytes)
                                         ? (size_t)kStages * kStageBytes : (kMergeBytes + 1023) / 1024 * 1024;
   static constexpr size_t kSmem = 1024 + kRegion + 2 * kStages * 8 + 16 + kPreTiles * kTile * 4;
@@ -218,10 +218,7 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
   float *ws_o = reinterpret_cast<float *>(stages);      // [warp][16][OS]
   float *ws_ml = ws_o + C::kWarps * 16 * OS;            // [warp][16][2]
   float *cpart = ws_ml + C::kWarps * 16 * 2;            // [H][kPartRow]: this CTA's (M, L, O)
-  {
-    const float f[2] = {st.vref, st.vref};
-    o_to_smem<KV>(ws_o + warp * 16 * OS, st.o, f, true);
-  }
+  float *hml = cpart + H * kPartRow;                    // [H][2]: (M, L) of each head
   if (c == 0) {
     ws_ml[(warp * 16 + g) * 2 + 0] = st.m[0];
     ws_ml[(warp * 16 + g) * 2 + 1] = st.l[0];
@@ -229,32 +226,62 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
     ws_ml[(warp * 16 + g + 8) * 2 + 1] = st.l[1];
   }
   __syncthreads();
-  for (int t = threadIdx.x; t < H * kHeadDim; t += C::kThreads) {
-    const int h = t / kHeadDim, d = t % kHeadDim;
-    const int hgh = h >> 4, rh = h & 15;
-    float M = -INFINITY;
+  {  // each warp stores its output rows rescaled to the common maximum of their head
+    float f[2];
 #pragma unroll
-    for (int k = 0; k < TG; ++k) M = fmaxf(M, ws_ml[((k * HG + hgh) * 16 + rh) * 2]);
-    float L = 0.f, O = 0.f;
+    for (int hh = 0; hh < 2; ++hh) {
+      const int rw = g + 8 * hh;
+      float M = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < TG; ++k) M = fmaxf(M, ws_ml[((k * HG + hg) * 16 + rw) * 2]);
+      f[hh] = (st.m[hh] == -INFINITY) ? 0.f : fast_exp2(st.m[hh] - M) * st.vref;
+    }
+    o_to_smem<KV>(ws_o + warp * 16 * OS, st.o, f, true);
+    if (warp == 0) {   // (M, L) per head
+      const int h = lane, hgh = h >> 4, rh = h & 15;
+      if (h < H) {
+        float M = -INFINITY, L = 0.f;
+#pragma unroll
+        for (int k = 0; k < TG; ++k) M = fmaxf(M, ws_ml[((k * HG + hgh) * 16 + rh) * 2]);
+#pragma unroll
+        for (int k = 0; k < TG; ++k) {
+          const float m = ws_ml[((k * HG + hgh) * 16 + rh) * 2];
+          if (m != -INFINITY) L += fast_exp2(m - M) * ws_ml[((k * HG + hgh) * 16 + rh) * 2 + 1];
+        }
+        hml[2 * h] = M;
+        hml[2 * h + 1] = L;
+      }
+    }
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < H * kHeadDim / 4; t += C::kThreads) {   // sum of the token groups
+    const int h = t / (kHeadDim / 4), d4 = t % (kHeadDim / 4);
+    const int hgh = h >> 4, rh = h & 15;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < TG; ++k) {
-      const int w = k * HG + hgh;
-      const float m = ws_ml[(w * 16 + rh) * 2];
-      const float f = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
-      L += f * ws_ml[(w * 16 + rh) * 2 + 1];
-      O += f * ws_o[(w * 16 + rh) * OS + d];
+      const float4 o = reinterpret_cast<const float4 *>(ws_o + ((k * HG + hgh) * 16 + rh) * OS)[d4];
+      O.x += o.x;
+      O.y += o.y;
+      O.z += o.z;
+      O.w += o.w;
     }
     if (P.n_tsplit == 1) {
-      const float val = O / L;
-      const size_t oi = ((size_t)r * H + h) * kHeadDim + d;
-      if (P.out_f32) reinterpret_cast<float *>(P.out)[oi] = val;
-      else reinterpret_cast<__nv_bfloat16 *>(P.out)[oi] = __float2bfloat16_rn(val);
+      const float inv = 1.f / hml[2 * h + 1];
+      const size_t oi = ((size_t)r * H + h) * kHeadDim + 4 * d4;
+      if (P.out_f32) {
+        *reinterpret_cast<float4 *>(reinterpret_cast<float *>(P.out) + oi) =
+            make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+      } else {
+        *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(P.out) + oi) =
+            make_uint2(pack_bf16(O.x * inv, O.y * inv), pack_bf16(O.z * inv, O.w * inv));
+      }
     } else {
       float *row = cpart + h * kPartRow;
-      row[kPartO + d] = O;
-      if (d == 0) {
-        row[0] = M;
-        row[1] = L;
+      reinterpret_cast<float4 *>(row + kPartO)[d4] = O;
+      if (d4 == 0) {
+        row[0] = hml[2 * h];
+        row[1] = hml[2 * h + 1];
       }
     }
   }
@@ -428,6 +455,7 @@ int max_cluster_t() {
 }
 
 }  // namespace
+
 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t s) {
   cudaError_t e = launch_pdl(merge_partials_kernel, p.n_groups * p.n_heads * kMergeChunks, kMergeThreads, 0, s, p);
