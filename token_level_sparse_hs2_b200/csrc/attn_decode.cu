@@ -30,7 +30,8 @@ namespace {
 // 8 consumer warps in one CTA per SM; pass 2 runs 4 in each of two CTAs per SM.
 template <int KV, int HG, int PASS>
 struct StreamCfg {
-  static constexpr int kGroupWarps = (PASS == 0) ? 4 * HG : 4;
+  static constexpr int kPass1Rows = 32;   // tile rows per pass-1 warp (NT = 4 n8 tiles)
+  static constexpr int kGroupWarps = (PASS == 0) ? (kTile / kPass1Rows) * HG : 4;
   static constexpr int kGroups = (PASS == 0) ? 8 / kGroupWarps : 1;
   static constexpr int kConsumers = kGroupWarps * kGroups;
   static constexpr int kThreads = (kConsumers + 1) * 32;
@@ -271,7 +272,8 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, 1)
   }
   const int grp = warp / C::kGroupWarps, gw = warp % C::kGroupWarps;
   const int hg = gw % HG, tg = gw / HG;
-  const int tok0 = tg * 16;
+  constexpr int NT = C::kPass1Rows / 8;
+  const int tok0 = tg * C::kPass1Rows;
   const int c = lane & 3;
   TileWalk wk(P, false);
   int cur = -1;
@@ -303,10 +305,10 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, 1)
     const uint8_t *stg = sm.stages + s * C::kStageBytes;
     const int64_t trow = tile_row0(P, b, g);
     const int64_t row0 = P.seq.start[b], row1 = row0 + P.seq.len[b];
-    bool valid[2][2];
-    float colk[2][2], colv[2][2];
+    bool valid[NT][2];
+    float colk[NT][2], colv[NT][2];
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int rr = tok0 + n * 8 + 2 * c + e;
@@ -321,9 +323,9 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, 1)
           colv[n][e] = 1.f;
         }
       }
-    float sacc[2][4];
-    qk_tile<KV, 2>(qa, smem_u32(stg), tok0, sacc);
-    softmax_pv_tile<KV, 2>(st, sacc, rowf, colk, colv, valid, smem_u32(stg + C::kKBytes), tok0);
+    float sacc[NT][4];
+    qk_tile<KV, NT>(qa, smem_u32(stg), tok0, sacc);
+    softmax_pv_tile<KV, NT>(st, sacc, rowf, colk, colv, valid, smem_u32(stg + C::kKBytes), tok0);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
   }
