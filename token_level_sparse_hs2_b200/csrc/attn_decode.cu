@@ -27,12 +27,17 @@ namespace {
 
 // Consumer warps come in groups that take turns on tiles (group i handles steps i, i + kGroups,
 // ...); within a group, pass-1 warps split heads x rows, pass-2 warps split rows. Pass 1 runs
-// 8 consumer warps in one CTA per SM; pass 2 runs 4 in each of two CTAs per SM.
+// 6 (bf16) or 8 (e4m3) consumer warps in one CTA per SM; pass 2 runs 4 in each of two CTAs
+// per SM.
 template <int KV, int HG, int PASS>
 struct StreamCfg {
-  static constexpr int kPass1Rows = 32;   // tile rows per pass-1 warp (NT = 4 n8 tiles)
-  static constexpr int kGroupWarps = (PASS == 0) ? (kTile / kPass1Rows) * HG : 4;
-  static constexpr int kGroups = (PASS == 0) ? 8 / kGroupWarps : 1;
+  // tile rows per pass-1 warp and pass-1 consumer warps: bf16 64 rows x 6 warps (registers
+  // for a whole tile's scores); e4m3 32 rows x 8 warps (the widening wants more warps)
+  static constexpr int kPass1Rows = (KV == kKvBf16) ? 64 : 32;
+  static constexpr int kPass1Warps = (KV == kKvBf16) ? 6 : 8;
+  static constexpr int kPass2Rows = 32;   // tile rows per pass-2 warp (all heads)
+  static constexpr int kGroupWarps = (PASS == 0) ? (kTile / kPass1Rows) * HG : kTile / kPass2Rows;
+  static constexpr int kGroups = (PASS == 0) ? kPass1Warps / kGroupWarps : 4 / kGroupWarps;
   static constexpr int kConsumers = kGroupWarps * kGroups;
   static constexpr int kThreads = (kConsumers + 1) * 32;
   static constexpr int kKBytes = (KV == kKvBf16) ? 2 * kBoxBytes : kBoxBytes;
@@ -362,7 +367,8 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, 2)
   } else {
     const int grp = warp / C::kGroupWarps, gw = warp % C::kGroupWarps;
     const int g8 = lane >> 2, c = lane & 3;
-    const int tok0 = gw * 16;
+    constexpr int NT2 = C::kPass2Rows / 8;
+    const int tok0 = gw * C::kPass2Rows;
     int cur = -1;
     int64_t n_cand = 0;
     uint32_t *hrow = nullptr;
@@ -395,22 +401,24 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, 2)
       const uint8_t *stg = sm.stages + s * C::kStageBytes;
       const int64_t trow = tile_row0(P, b, g);
       const int64_t row0 = P.seq.start[b], row1 = row0 + P.seq.len[b];
-      float colk[2][2];
+      float colk[NT2][2];
 #pragma unroll
-      for (int n = 0; n < 2; ++n)
+      for (int n = 0; n < NT2; ++n)
 #pragma unroll
         for (int e = 0; e < 2; ++e)
           colk[n][e] = (KV == kKvFp8)
                            ? reinterpret_cast<const float *>(stg + C::kKBytes)[tok0 + n * 8 + 2 * c + e]
                            : 1.f;
-      float sacc[HG][2][4];
-      qk_tile_mt<KV, HG, 2>(qa, smem_u32(stg), tok0, sacc);
+      float sacc[HG][NT2][4];
+      qk_tile_mt<KV, HG, NT2>(qa, smem_u32(stg), tok0, sacc);
       // x = s * (rowf * colk) - lse2 and the sum over heads, two columns at a time
-      float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float2 acc[NT2];
+#pragma unroll
+      for (int n = 0; n < NT2; ++n) acc[n] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int mt = 0; mt < HG; ++mt)
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+        for (int n = 0; n < NT2; ++n)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const float2 a = make_float2(rowf[mt][h] * colk[n][0], rowf[mt][h] * colk[n][1]);
@@ -418,11 +426,16 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, 2)
                                    make_float2(-lse2[mt][h], -lse2[mt][h]));
             acc[n] = fadd2(acc[n], make_float2(fast_exp2(x.x), fast_exp2(x.y)));
           }
-      float cs[2][2] = {{acc[0].x, acc[0].y}, {acc[1].x, acc[1].y}};
+      float cs[NT2][2];
+#pragma unroll
+      for (int n = 0; n < NT2; ++n) {
+        cs[n][0] = acc[n].x;
+        cs[n][1] = acc[n].y;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
 #pragma unroll
-      for (int n = 0; n < 2; ++n)
+      for (int n = 0; n < NT2; ++n)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           float v = cs[n][e];
@@ -434,7 +447,7 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, 2)
       if (g8 == 0) {
         float *srow = P.scores + (size_t)b * P.score_stride;
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+        for (int n = 0; n < NT2; ++n)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int64_t row = trow + tok0 + n * 8 + 2 * c + e;
