@@ -160,7 +160,7 @@ def dist_setup(a):
     return world, rank, local
 
 
-def cpu_baseline(w, budget_s=20.0):
+def cpu_baseline(w, budget_s=12.0):
     """The oracle as it stands, on the host cores, over whole batches of the same workload."""
     import oracle
     oracle.build()
@@ -170,7 +170,7 @@ def cpu_baseline(w, budget_s=20.0):
         oracle.block(w, rows=rows)
         reps += 1
         el = time.perf_counter() - t0
-        if el > budget_s * 0.5 or reps >= 3:
+        if el > budget_s or reps >= 200:
             break
     tok = reps * w.n_rows
     return {"value": tok / el, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
