@@ -153,6 +153,21 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def slowest(x: float, dist=None, device=None) -> float:
+    """The largest x over the ranks (the slowest rank's time); x itself without a process group.
+    The reduction runs on `device` (CUDA for NCCL, CPU for gloo)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(units_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job rate: every rank's units over the slowest rank's time (weak scaling)."""
+    return world * units_per_rank / (ms / 1e3)
+
+
 def dist_setup(a):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -273,10 +288,7 @@ def main():
     barrier()
     hs2.read_device_status(ws)
     ms = t_start.elapsed_time(t_end) / a.steps
-    ms_t = torch.tensor([ms], device=dev)
-    if pg:
-        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = slowest(ms, pg, dev)
 
     # ---- the same K steps again with an event between consecutive kernels (per-kernel times;
     # the events break the programmatic-launch overlap, so this step time runs a little longer)
@@ -334,12 +346,10 @@ def main():
         a1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = torch.tensor([a0.elapsed_time(a1) / a.steps], device=dev)
-        if pg:
-            pg.all_reduce(ems, op=pg.ReduceOp.MAX)
-        e2e = {"value": world * R / (float(ems.item()) / 1e3), "unit": UNIT,
+        ems = slowest(a0.elapsed_time(a1) / a.steps, pg, dev)
+        e2e = {"value": throughput(R, world, ems), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": float(ems.item())}
+               "ms_per_step": ems}
 
     hbm, tf_burst, tf_sust, how = peaks()
     ab = algorithmic_bytes(w)
@@ -371,7 +381,7 @@ def main():
             "frac": a2 / tf_sust, "frac_of_burst_peak": a2 / tf_burst,
             "flops_per_launch": fl["pass2"], "ms_per_launch": per["pass2"]}}
     line = {
-        "metric": METRIC, "value": world * R / (ms_max / 1e3), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": throughput(R, world, ms_max), "unit": UNIT, "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms_max, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.kv_dtype == "bf16" else "fp8-e4m3 (bf16/f16 math)",
