@@ -191,6 +191,15 @@ const char *hs2_last_error(void);
 const char *hs2_status_string(hs2_status status);
 int32_t hs2_version(void);
 
+/* Exercises the bounded waits of the kernels: one thread waits on an mbarrier that nothing
+ * arrives at, gives up after limit_us microseconds (1 .. 2e6) and records HS2_ERR_TIMEOUT in the
+ * status word at the start of `workspace` (device, 256-byte aligned, >= 256 bytes), which the
+ * call clears first; hs2_read_device_status then reports HS2_ERR_TIMEOUT and the context stays
+ * usable. Not part of the method: a failure-detection check. Returns HS2_ERR_WORKSPACE /
+ * HS2_ERR_INVALID_ARG on bad arguments (nothing launched), HS2_ERR_CUDA on a launch error. */
+hs2_status hs2_selftest_wait_timeout(uint32_t limit_us, void *workspace, size_t workspace_bytes,
+                                     void *stream);
+
 /* Number of kernels this library has launched in the calling process since it was loaded
  * (successful launches only; the workspace clears done with cudaMemsetAsync are not counted).
  * Not part of the method: an accounting aid for callers that count launches per call. */

@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.hs2_status_string.argtypes = [ctypes.c_int]
         L.hs2_version.restype = I32
         L.hs2_launch_count.restype = ctypes.c_uint64
+        L.hs2_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P, SZ, P]
+        L.hs2_selftest_wait_timeout.restype = ctypes.c_int
         for name in ("hs2_workspace_size", "hs2_full_attn_scores", "hs2_topk_select",
                      "hs2_sparse_gather_attn", "hs2_block_decode", "hs2_block_decode_traced",
                      "hs2_topk_select_noalloc", "hs2_read_device_status"):
@@ -242,3 +244,12 @@ def read_device_status(workspace, stream=None):
 def launch_count() -> int:
     """Kernels the library has launched in this process so far (hs2_launch_count)."""
     return int(lib().hs2_launch_count())
+
+
+def selftest_wait_timeout(workspace, limit_us: int = 20000, stream=None):
+    """Runs hs2_selftest_wait_timeout: a kernel whose bounded wait must run out; returns the
+    status hs2_read_device_status then reports (an int, HS2_ERR_TIMEOUT = 6 expected)."""
+    _check(lib().hs2_selftest_wait_timeout(limit_us, _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(),
+                                          _stream(stream)))
+    return int(lib().hs2_read_device_status(_ptr(workspace), _stream(stream)))

@@ -16,6 +16,7 @@
 #include <functional>
 #include <mutex>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace hs2 {
@@ -782,6 +783,35 @@ hs2_status hs2_read_device_status(const void *workspace, void *stream) {
   if (st != HS2_OK) return st;
   if (v & kStatusTimeout) return fail(HS2_ERR_TIMEOUT, "a kernel's bounded wait ran out");
   if (v & kStatusCheck) return fail(HS2_ERR_DEVICE_CHECK, "a kernel found an out-of-range index or count");
+  return ok();
+}
+
+namespace hs2 {
+namespace {
+// One thread waits, bounded by limit_ns, on an mbarrier that expects one arrival and gets none,
+// and records the timeout in the status word like every kernel of the library does.
+__global__ void selftest_wait_kernel(uint32_t *status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+    if (!mbar_wait_for(smem_u32(&bar), 0, limit_ns)) record_status(status, kStatusTimeout);
+  }
+}
+}  // namespace
+}  // namespace hs2
+
+hs2_status hs2_selftest_wait_timeout(uint32_t limit_us, void *workspace, size_t workspace_bytes,
+                                     void *stream) {
+  if (!workspace || workspace_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(HS2_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold 256 bytes");
+  if (limit_us < 1 || limit_us > 2000000) return fail(HS2_ERR_INVALID_ARG, "limit_us %u outside [1, 2e6]", limit_us);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  hs2_status st = cuda_check(cudaMemsetAsync(workspace, 0, 4, s), "status clear");
+  if (st != HS2_OK) return st;
+  hs2::selftest_wait_kernel<<<1, 32, 0, s>>>(static_cast<uint32_t *>(workspace), (uint64_t)limit_us * 1000ull);
+  if ((st = cuda_check(cudaGetLastError(), "self-test launch")) != HS2_OK) return st;
+  hs2::note_launch();
   return ok();
 }
 
