@@ -307,13 +307,23 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < ns; ++j) {
-      const float f = __shfl_sync(0xffffffffu, fj, j);
-      const float4 o = reinterpret_cast<const float4 *>(cluster.map_shared_rank(cpart, j) + h * kPartRow + kPartO)[lane];
-      O.x += f * o.x;
-      O.y += f * o.y;
-      O.z += f * o.z;
-      O.w += f * o.w;
+    for (int j0 = 0; j0 < ns; j0 += 4) {   // four remote loads in flight at a time
+      float4 o[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        o[u] = (j0 + u < ns)
+                   ? reinterpret_cast<const float4 *>(cluster.map_shared_rank(cpart, j0 + u) + h * kPartRow + kPartO)[lane]
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float f = __shfl_sync(0xffffffffu, fj, (j0 + u) & 31);
+        if (j0 + u < ns) {
+          O.x += f * o[u].x;
+          O.y += f * o[u].y;
+          O.z += f * o[u].z;
+          O.w += f * o[u].w;
+        }
+      }
     }
     const float inv = 1.f / L;
     const size_t oi = ((size_t)r * H + h) * kHeadDim + 4 * lane;
