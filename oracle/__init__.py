@@ -69,6 +69,9 @@ def lib():
         L.hs2o_sparse_attn.argtypes = [P, P, D, P, I64, P, I64, P, P]
         L.hs2o_sparse_attn.restype = I32
         L.hs2o_num_threads.restype = I32
+        L.hs2o_e4m3_rne.argtypes = [ctypes.c_float]
+        L.hs2o_e4m3_rne.restype = ctypes.c_uint8
+        L.hs2o_quantize_row.argtypes = [P, I32, P, P]
         _lib = L
     return _lib
 
@@ -210,3 +213,20 @@ def block(w, rows=None, scale=None):
                 for l in range(w.n_sparse)]
     return dict(rows=rows, o_full=o_full, lse=lse, scores=s, idx=idx, count=count,
                 o_sparse=o_sparse)
+
+
+def e4m3_rne(y: float) -> int:
+    """OCP e4m3fn code nearest to the float32 value y (ties to even, saturating at 448)."""
+    return int(lib().hs2o_e4m3_rne(float(y)))
+
+
+def quantize_rows(x_bf16_bits: np.ndarray):
+    """FP8 cache rows for appended tokens: x as bf16 bits [rows, d] -> (codes uint8 [rows, d],
+    scale float32 [rows]); scale = max|x| / 448 (1 for a zero row), codes = e4m3 RNE of x / scale."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    rows, d = x.shape
+    codes = np.zeros((rows, d), dtype=np.uint8)
+    scale = np.zeros(rows, dtype=np.float32)
+    for r in range(rows):
+        lib().hs2o_quantize_row(x[r].ctypes.data, d, codes[r].ctypes.data, scale[r:].ctypes.data)
+    return codes, scale

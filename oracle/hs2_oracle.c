@@ -340,3 +340,53 @@ int hs2o_num_threads(void) {
   return 1;
 #endif
 }
+
+/* ---------------------------------------------------------------- KV append (FP8 quantise) */
+
+/* Round-to-nearest-even of y (|y| <= 448, already a float32 value) to the OCP e4m3fn code,
+ * from the format definition: subnormals are multiples of 2^-9 below 2^-6; a normal value with
+ * exponent e in [-6, 8] has mantissa steps of 2^(e-3); a carry out of the mantissa moves to the
+ * next exponent; the largest finite value 448 (S.1111.110) is the saturation point. */
+uint8_t hs2o_e4m3_rne(float y) {
+  const int neg = signbit(y) ? 1 : 0;
+  double a = fabs((double)y);
+  if (a > 448.0) a = 448.0;
+  int code;
+  if (a < ldexp(1.0, -6)) {
+    code = (int)rint(a / ldexp(1.0, -9));          /* 0..8; 8 is the smallest normal (0x08) */
+  } else {
+    int e;
+    frexp(a, &e);                                     /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;                                           /* a = (1 + frac) * 2^e */
+    int q = (int)rint((a / ldexp(1.0, e) - 1.0) * 8.0);
+    int E = e + 7;
+    if (q == 8) {
+      q = 0;
+      E += 1;
+    }
+    code = (E << 3) | q;
+    if (code > 0x7e) code = 0x7e;
+  }
+  return (uint8_t)(code | (neg << 7));
+}
+
+/* The FP8 cache write of one appended row of d bf16 values: scale = max|x| / 448 in float32
+ * (1 for an all-zero row), codes = e4m3 RNE of the float32 quotient x / scale, saturated at 448. */
+void hs2o_quantize_row(const uint16_t *x_bf16, int d, uint8_t *codes, float *scale) {
+  float amax = 0.f;
+  for (int j = 0; j < d; ++j) {
+    uint32_t u = (uint32_t)x_bf16[j] << 16;
+    float v;
+    memcpy(&v, &u, 4);
+    if (fabsf(v) > amax) amax = fabsf(v);
+  }
+  const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
+  for (int j = 0; j < d; ++j) {
+    uint32_t u = (uint32_t)x_bf16[j] << 16;
+    float v;
+    memcpy(&v, &u, 4);
+    const float y = v / sc;
+    codes[j] = hs2o_e4m3_rne(y);
+  }
+  *scale = sc;
+}

@@ -262,3 +262,55 @@ def test_planted_mistake_is_caught(oracle_lib):
     assert np.array_equal(got, ref)
     wrong = np.sort(np.lexsort((np.arange(p + 1), -s))[:k + win])   # window not forced
     assert not np.array_equal(wrong, ref)
+
+
+# ------------------------------------------------------------------ KV append: FP8 quantiser
+# "HySparse2: Hybrid Sparse Attention with Two-Level KV Sharing", "Inference cost": the shared
+# KV cache is FP8; appended rows are quantised per token (scale = max|x| / 448, e4m3 RNE).
+
+def test_e4m3_rne_matches_torch_cast(oracle_lib):
+    rng = np.random.default_rng(7)
+    ys = np.concatenate([rng.uniform(-448, 448, 20000), rng.normal(0, 1e-2, 20000),
+                         rng.normal(0, 3e-3, 5000), [0.0, -0.0, 448.0, -448.0, 2.0 ** -9, 2.0 ** -10]])
+    ys = ys.astype(np.float32)
+    ref = torch.from_numpy(ys).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle_lib.e4m3_rne(float(y)) for y in ys], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_rne_round_trips_every_code_and_ties_go_to_even(oracle_lib):
+    table = oracle_lib.e4m3_table()
+    finite = [c for c in range(256) if not np.isnan(table[c])]
+    for c in finite:
+        assert oracle_lib.e4m3_rne(float(table[c])) == c
+    pos = sorted(c for c in finite if c < 0x80)           # ascending magnitudes 0 .. 448
+    for a, b in zip(pos[:-1], pos[1:]):
+        mid = np.float32((table[a] + table[b]) / 2)
+        if float(mid) != (table[a] + table[b]) / 2:
+            continue                                     # not exactly representable in float32
+        even = a if a % 2 == 0 else b
+        assert oracle_lib.e4m3_rne(float(mid)) == even
+    assert oracle_lib.e4m3_rne(1000.0) == 0x7e and oracle_lib.e4m3_rne(-1000.0) == 0xfe
+
+
+def test_quantize_rows_scale_codes_and_error_bound(oracle_lib):
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((64, 128)).astype(np.float32) * rng.uniform(0.01, 50, (64, 1)).astype(np.float32)
+    x[3] = 0.0
+    x[5, :] = 0.0
+    x[5, 17] = -2.5
+    bits = W.f32_to_bf16_bits(x)
+    xf = W.bf16_bits_to_f32(bits)
+    codes, scale = oracle_lib.quantize_rows(bits)
+    amax = np.abs(xf).max(axis=1)
+    assert scale[3] == 1.0 and not codes[3].any()
+    np.testing.assert_array_equal(scale[amax > 0], (amax[amax > 0] / np.float32(448.0)).astype(np.float32))
+    table = oracle_lib.e4m3_table()
+    deq = table[codes] * scale[:, None].astype(np.float64)
+    # the largest element of each row maps to +-448 exactly; every element within half a step
+    big = np.abs(xf).argmax(axis=1)
+    assert np.all(np.abs(table[codes[np.arange(64), big]])[amax > 0] == 448.0)
+    err = np.abs(deq - xf)
+    step = np.maximum(np.abs(xf) / 8.0, 2.0 ** -9 * scale[:, None])    # 3 mantissa bits; subnormal floor
+    assert np.all(err <= step * 0.5 + 1e-12)
+    assert codes[5, 17] == 0xfe and np.all(codes[5, np.arange(128) != 17] == 0)
