@@ -219,6 +219,32 @@ def run_reference(a, w):
     print(json.dumps(line), flush=True)
 
 
+def bench_kv_append(hs2, dev, hbm, rows=65536, iters=20):
+    """The cache append (the step before the block) on a bulk of rows into an e4m3 cache: bytes
+    = rows x (K and V: 256 B read, 128 B codes + 4 B scale written), over the event time."""
+    k = torch.zeros((rows, 128), dtype=torch.uint8, device=dev)
+    v = torch.zeros_like(k)
+    ks = torch.zeros(rows, dtype=torch.float32, device=dev)
+    vs = torch.zeros_like(ks)
+    cache = hs2.KvCache(k, v, [0], [rows], rows, 32, ks, vs)
+    nk = torch.randn((1, rows, 128), device=dev).to(torch.bfloat16)
+    nv = torch.randn((1, rows, 128), device=dev).to(torch.bfloat16)
+    for _ in range(3):
+        hs2.kv_append(cache, nk, nv)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(iters):
+        hs2.kv_append(cache, nk, nv)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / iters * 1e3
+    nbytes = rows * 2 * (256 + 128 + 4)
+    gbs = nbytes / (us / 1e6) / 1e9
+    return {"kernel": "kv_append_kernel", "rows": rows, "kv_dtype": "fp8-e4m3", "us": us,
+            "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm}
+
+
 def config_of(w):
     return {"workload": w.name, "batch": w.batch, "queries_per_seq": w.n_q,
             "context_tokens_total": int(w.kv_len.astype(np.int64).sum()),
@@ -400,6 +426,7 @@ def main():
     }
     if e2e:
         line["e2e"] = e2e
+    line["kv_append"] = bench_kv_append(hs2, dev, hbm)
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

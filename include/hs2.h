@@ -191,6 +191,19 @@ const char *hs2_last_error(void);
 const char *hs2_status_string(hs2_status status);
 int32_t hs2_version(void);
 
+/* Appends the n_q new tokens of every sequence to the shared cache ("HySparse2: Hybrid Sparse
+ * Attention with Two-Level KV Sharing", "Inference cost": one FP8 K/V head shared by all query
+ * heads; the step before the block, since the window and the sparse layers read this cache).
+ * Cache row kv_start[b] + kv_len[b] - n_q + i (the sequence's last n_q rows, which kv_len
+ * already counts) receives new_k[b][i][:] and new_v[b][i][:] (device, bf16 [batch, n_q, 128],
+ * 16-byte aligned). bf16 cache: copied. e4m3 cache: per row and matrix, scale = max|x| / 448 in
+ * float32 (1 for an all-zero row) is written to k_scale / v_scale and the codes are the
+ * round-to-nearest-even e4m3 of x * (1 / scale) (the reciprocal rounded to float32), saturated
+ * at 448. The view's K/V (and scale) buffers
+ * are written: they are caller-owned device memory. Asynchronous on `stream`; argument errors
+ * return before any launch. */
+hs2_status hs2_kv_append(const hs2_kv_view *kv, const void *new_k, const void *new_v, void *stream);
+
 /* Exercises the bounded waits of the kernels: one thread waits on an mbarrier that nothing
  * arrives at, gives up after limit_us microseconds (1 .. 2e6) and records HS2_ERR_TIMEOUT in the
  * status word at the start of `workspace` (device, 256-byte aligned, >= 256 bytes), which the

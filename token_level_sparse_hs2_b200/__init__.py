@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.hs2_version.restype = I32
         L.hs2_launch_count.restype = ctypes.c_uint64
         L.hs2_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P, SZ, P]
+        L.hs2_kv_append.argtypes = [V, P, P, P]
+        L.hs2_kv_append.restype = ctypes.c_int
         L.hs2_selftest_wait_timeout.restype = ctypes.c_int
         for name in ("hs2_workspace_size", "hs2_full_attn_scores", "hs2_topk_select",
                      "hs2_sparse_gather_attn", "hs2_block_decode", "hs2_block_decode_traced",
@@ -253,3 +255,9 @@ def selftest_wait_timeout(workspace, limit_us: int = 20000, stream=None):
                                           workspace.numel() * workspace.element_size(),
                                           _stream(stream)))
     return int(lib().hs2_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+def kv_append(cache: KvCache, new_k, new_v, stream=None):
+    """Writes the n_q new tokens of every sequence (bf16 [batch, n_q, 128] each) into the last
+    n_q rows of each sequence of the cache (e4m3 caches: quantised with per-row scales)."""
+    _check(lib().hs2_kv_append(cache.ref(), _ptr(new_k), _ptr(new_v), _stream(stream)))

@@ -801,6 +801,31 @@ __global__ void selftest_wait_kernel(uint32_t *status, uint64_t limit_ns) {
 }  // namespace
 }  // namespace hs2
 
+hs2_status hs2_kv_append(const hs2_kv_view *kv, const void *new_k, const void *new_v, void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if (!new_k || !new_v) return fail(HS2_ERR_INVALID_ARG, "new_k / new_v is NULL");
+  if ((reinterpret_cast<uintptr_t>(new_k) | reinterpret_cast<uintptr_t>(new_v)) & 15)
+    return fail(HS2_ERR_INVALID_ARG, "new_k / new_v must be 16-byte aligned");
+  hs2::AppendParams ap;
+  memset(&ap, 0, sizeof ap);
+  for (int b = 0; b < kv->batch; ++b) {
+    ap.seq.start[b] = kv->kv_start[b];
+    ap.seq.len[b] = kv->kv_len[b];
+  }
+  ap.batch = kv->batch;
+  ap.n_q = kv->n_q;
+  ap.fp8 = kv->kv_dtype == HS2_KV_FP8_E4M3;
+  ap.new_k = new_k;
+  ap.new_v = new_v;
+  ap.k = const_cast<void *>(kv->k);
+  ap.v = const_cast<void *>(kv->v);
+  ap.k_scale = const_cast<float *>(kv->k_scale);
+  ap.v_scale = const_cast<float *>(kv->v_scale);
+  st = cuda_check(hs2::launch_kv_append(ap, static_cast<cudaStream_t>(stream)), "kv append");
+  return st == HS2_OK ? ok() : st;
+}
+
 hs2_status hs2_selftest_wait_timeout(uint32_t limit_us, void *workspace, size_t workspace_bytes,
                                      void *stream) {
   if (!workspace || workspace_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 255))

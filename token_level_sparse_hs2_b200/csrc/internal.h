@@ -102,6 +102,16 @@ struct SparseParams {
   uint32_t *status;
 };
 
+// Cache append of n_q new rows per sequence (the last n_q rows of each sequence).
+struct AppendParams {
+  SeqTable seq;
+  int32_t batch, n_q, fp8;
+  const void *new_k, *new_v;  // bf16 [B, n_q, 128]
+  void *k, *v;                // cache rows (bf16 or e4m3)
+  float *k_scale, *v_scale;   // e4m3: per-row scales
+};
+cudaError_t launch_kv_append(const AppendParams &p, cudaStream_t s);
+
 // Largest thread-block cluster the sparse layer may use for this cache type and head count.
 int sparse_max_cluster(int kv_dtype, int n_heads);
 
