@@ -72,6 +72,14 @@ def lib():
         L.hs2o_e4m3_rne.argtypes = [ctypes.c_float]
         L.hs2o_e4m3_rne.restype = ctypes.c_uint8
         L.hs2o_quantize_row.argtypes = [P, I32, P, P]
+        L.hs2o_select_blocks_f64.argtypes = [P, I64, I32, I32, I32, P]
+        L.hs2o_select_blocks_f64.restype = I64
+        L.hs2o_select_blocks_f32.argtypes = [P, I64, I32, I32, I32, P]
+        L.hs2o_select_blocks_f32.restype = I64
+        L.hs2o_block_score_f32.argtypes = [P, I64, I64, I32]
+        L.hs2o_block_score_f32.restype = ctypes.c_float
+        L.hs2o_select_blocks_rows.argtypes = [P, P, I64, P, I64, I32, I32, I32, I32, P, I64, P]
+        L.hs2o_select_blocks_rows.restype = I32
         _lib = L
     return _lib
 
@@ -182,6 +190,52 @@ def select_rows(w, rows, scores, topk=None, window=None, fp32=False):
                                         count.ctypes.data)
     if rc != 0:
         raise RuntimeError("oracle select failed")
+    return out, count
+
+
+def select_blocks_f64(s: np.ndarray, p: int, block: int, topk: int, window: int) -> np.ndarray:
+    """Block-level selection (blocks of `block` candidate positions, block score = sum)."""
+    s = np.ascontiguousarray(s, dtype=np.float64)
+    out = np.empty(max(p + 1, 1), dtype=np.int32)
+    c = lib().hs2o_select_blocks_f64(s.ctypes.data, p, block, topk, window, out.ctypes.data)
+    if c < 0:
+        raise ValueError("block size must be a power of two dividing topk")
+    return out[:c]
+
+
+def select_blocks_f32(s: np.ndarray, p: int, block: int, topk: int, window: int) -> np.ndarray:
+    """Block-level selection on float32 scores (fold-in-half float32 block sums)."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    out = np.empty(max(p + 1, 1), dtype=np.int32)
+    c = lib().hs2o_select_blocks_f32(s.ctypes.data, p, block, topk, window, out.ctypes.data)
+    if c < 0:
+        raise ValueError("block size must be a power of two dividing topk (at most 4096)")
+    return out[:c]
+
+
+def block_score_f32(s: np.ndarray, t0: int, nc: int, block: int) -> float:
+    """float32 score of the block starting at t0 (positions >= nc count as 0)."""
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    return float(lib().hs2o_block_score_f32(s.ctypes.data, t0, nc, block))
+
+
+def select_blocks_rows(w, rows, scores, block, topk=None, window=None, fp32=False):
+    """Block-level selection for listed rows; returns (idx [n, cap], count) like select_rows."""
+    topk = w.topk if topk is None else topk
+    window = w.window if window is None else window
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    n = rows.size
+    cap = max(int(positions(w, rows).max()) + 1 if n else 1, 1)
+    cap = min(cap, topk + window)
+    out = np.full((n, cap), -1, dtype=np.int32)
+    count = np.zeros(n, dtype=np.int32)
+    view = _View(w)
+    s = np.ascontiguousarray(scores, dtype=np.float32 if fp32 else np.float64)
+    rc = lib().hs2o_select_blocks_rows(view.ref, rows.ctypes.data, n, s.ctypes.data, s.shape[1],
+                                       1 if fp32 else 0, block, topk, window, out.ctypes.data,
+                                       cap, count.ctypes.data)
+    if rc != 0:
+        raise RuntimeError("oracle block select failed")
     return out, count
 
 

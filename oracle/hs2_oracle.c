@@ -276,6 +276,124 @@ int hs2o_select_rows_f32(const hs2o_kv *kv, const int64_t *rows, int64_t n_rows,
   return bad ? -1 : 0;
 }
 
+/* ---------------------------------------------------------------- block-level selection */
+
+/* The block-granular selection HySparse used and HySparse2 replaces ("HySparse2: How Xiaomi
+ * Split the Transformer to Fix Agent Prefill Costs", section "KV Reuse and Token-Level Sparse
+ * Selection": block-level selection hands the budget out 64 tokens at a time; the token-level
+ * variant hands out the same 1,024 tokens one by one; "HySparse2: Hybrid Sparse Attention with
+ * Two-Level KV Sharing", bullet "KV Reuse refinements": same attention budget). Read here as:
+ * the candidates C = [0, nc) are cut at multiples of the block size bs into blocks
+ * [j*bs, min((j+1)*bs, nc)); a block's score is the sum of its candidates' scores; the
+ * topk / bs blocks with the largest score (ties: lower block index) are kept, their positions
+ * in ascending order, then the window W = [nc, p]. If nc <= topk every position is kept, as
+ * for tokens. bs must be a power of two that divides topk. */
+static int64_t select_blocks_common(cand_t *blk, int64_t nb, int64_t nc, int64_t p, int bs,
+                                    int topk, int window, int32_t *out) {
+  const int kb = topk / bs;
+  qsort(blk, (size_t)nb, sizeof(cand_t), cmp_cand);
+  int32_t *ids = (int32_t *)malloc(sizeof(int32_t) * (size_t)kb);
+  if (!ids) return -1;
+  for (int j = 0; j < kb; ++j) ids[j] = (int32_t)blk[j].t;
+  qsort(ids, (size_t)kb, sizeof(int32_t), cmp_i32);
+  int64_t cnt = 0;
+  for (int j = 0; j < kb; ++j) {
+    const int64_t t0 = (int64_t)ids[j] * bs;
+    const int64_t t1 = t0 + bs < nc ? t0 + bs : nc;
+    for (int64_t t = t0; t < t1; ++t) out[cnt++] = (int32_t)t;
+  }
+  free(ids);
+  for (int64_t t = nc; t <= p; ++t) out[cnt++] = (int32_t)t;
+  return cnt;
+}
+
+static int blocks_args_ok(int bs, int topk) {
+  return bs >= 1 && (bs & (bs - 1)) == 0 && topk >= bs && topk % bs == 0;
+}
+
+/* fp64 selector: block score = the block's candidate scores summed in double, in index order. */
+int64_t hs2o_select_blocks_f64(const double *s, int64_t p, int bs, int topk, int window,
+                               int32_t *out) {
+  if (!blocks_args_ok(bs, topk)) return -1;
+  int64_t nc = p - window + 1;
+  if (nc < 0) nc = 0;
+  if (nc <= topk) {
+    for (int64_t t = 0; t <= p; ++t) out[t] = (int32_t)t;
+    return p + 1;
+  }
+  const int64_t nb = (nc + bs - 1) / bs;
+  cand_t *blk = (cand_t *)malloc(sizeof(cand_t) * (size_t)nb);
+  if (!blk) return -1;
+  for (int64_t j = 0; j < nb; ++j) {
+    double acc = 0.0;
+    for (int64_t t = j * bs; t < (j + 1) * bs && t < nc; ++t) acc += s[t];
+    blk[j].key = acc;
+    blk[j].t = j;
+  }
+  int64_t cnt = select_blocks_common(blk, nb, nc, p, bs, topk, window, out);
+  free(blk);
+  return cnt;
+}
+
+/* The float32 block score: the bs values of the block (0 for positions >= nc) summed by folding
+ * the array in half until one value remains (v[i] = v[i] + v[i + n/2] for i < n/2, n = bs, bs/2,
+ * ..., 2), each addition rounded to float32. This fixed order makes the score -- and so the
+ * selection -- a function of the fp32 scores alone. */
+float hs2o_block_score_f32(const float *s, int64_t t0, int64_t nc, int bs) {
+  float v[4096];
+  if (bs < 1 || bs > 4096 || (bs & (bs - 1))) return -1.0f;
+  for (int i = 0; i < bs; ++i) v[i] = (t0 + i < nc) ? s[t0 + i] : 0.0f;
+  for (int n = bs; n > 1; n /= 2)
+    for (int i = 0; i < n / 2; ++i) v[i] = v[i] + v[i + n / 2];
+  return v[0];
+}
+
+/* fp32 selector (e.g. on the GPU's scores): block scores as hs2o_block_score_f32, ordered by
+ * their bit patterns (numeric order for non-negative floats). */
+int64_t hs2o_select_blocks_f32(const float *s, int64_t p, int bs, int topk, int window,
+                               int32_t *out) {
+  if (!blocks_args_ok(bs, topk) || bs > 4096) return -1;
+  int64_t nc = p - window + 1;
+  if (nc < 0) nc = 0;
+  if (nc <= topk) {
+    for (int64_t t = 0; t <= p; ++t) out[t] = (int32_t)t;
+    return p + 1;
+  }
+  const int64_t nb = (nc + bs - 1) / bs;
+  cand_t *blk = (cand_t *)malloc(sizeof(cand_t) * (size_t)nb);
+  if (!blk) return -1;
+  for (int64_t j = 0; j < nb; ++j) {
+    const float v = hs2o_block_score_f32(s, j * bs, nc, bs);
+    uint32_t u;
+    memcpy(&u, &v, sizeof u);
+    blk[j].key = (double)u;
+    blk[j].t = j;
+  }
+  int64_t cnt = select_blocks_common(blk, nb, nc, p, bs, topk, window, out);
+  free(blk);
+  return cnt;
+}
+
+/* Batched block selectors over listed rows (layouts as hs2o_select_rows_*); fp32 != 0 picks the
+ * float32 selector on float scores, else the fp64 one on double scores. */
+int hs2o_select_blocks_rows(const hs2o_kv *kv, const int64_t *rows, int64_t n_rows,
+                            const void *scores, int64_t score_stride, int fp32, int bs, int topk,
+                            int window, int32_t *out, int64_t out_stride, int32_t *count) {
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : bad)
+  for (int64_t rr = 0; rr < n_rows; ++rr) {
+    int64_t r = rows[rr], b = r / kv->n_q, i = r % kv->n_q;
+    int64_t p = (int64_t)kv->kv_len[b] - kv->n_q + i;
+    int64_t c = fp32 ? hs2o_select_blocks_f32((const float *)scores + rr * score_stride, p, bs,
+                                              topk, window, out + rr * out_stride)
+                     : hs2o_select_blocks_f64((const double *)scores + rr * score_stride, p, bs,
+                                              topk, window, out + rr * out_stride);
+    if (c < 0) bad = 1;
+    count[rr] = (int32_t)c;
+  }
+  return bad ? -1 : 0;
+}
+
 /* ---------------------------------------------------------------- sparse attention */
 
 /* For each listed row, attention of its own queries over the selected cache positions only:
