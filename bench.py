@@ -245,6 +245,44 @@ def bench_kv_append(hs2, dev, hbm, rows=65536, iters=20):
             "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm}
 
 
+def bench_block_select(hs2, cache, scores, w, dev, token_ms, block_size=64, iters=20):
+    """Block-level selection (HySparse's granularity at the same budget) on the step's own
+    scores, beside the token-level selection's traced time: pooling + per-row select."""
+    R = w.n_rows
+    cap = min(int(w.kv_len.max()), w.topk + w.window)
+    idx = torch.empty((R, cap), dtype=torch.int32, device=dev)
+    cnt = torch.empty(R, dtype=torch.int32, device=dev)
+    ws = torch.empty(hs2.topk_select_blocks_workspace_size(cache, block_size, w.topk, w.window),
+                     dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            hs2.topk_select_blocks(cache, scores, idx, cnt, ws, block_size, w.topk, w.window)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    # the calls are replayed from a CUDA graph so that the host's per-call cost does not show
+    n0 = hs2.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(iters):
+            hs2.topk_select_blocks(cache, scores, idx, cnt, ws, block_size, w.topk, w.window)
+    launches = (hs2.launch_count() - n0) / iters
+    graph.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del graph
+    return {"kernels": ["block_pool_kernel", "block_select_kernel"] if w.n_rows < 148
+            else ["block_select_kernel (pooling fused)"], "block_size": block_size,
+            "blocks_kept": w.topk // block_size, "us": e0.elapsed_time(e1) / iters * 1e3,
+            "launches_per_call": launches, "timing": "CUDA graph of %d calls" % iters,
+            "token_topk_us_traced": token_ms * 1e3}
+
+
 def config_of(w):
     return {"workload": w.name, "batch": w.batch, "queries_per_seq": w.n_q,
             "context_tokens_total": int(w.kv_len.astype(np.int64).sum()),
@@ -427,6 +465,7 @@ def main():
     if e2e:
         line["e2e"] = e2e
     line["kv_append"] = bench_kv_append(hs2, dev, hbm)
+    line["block_select"] = bench_block_select(hs2, cache, scores, w, dev, per["topk"])
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:

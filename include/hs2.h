@@ -182,6 +182,29 @@ hs2_status hs2_topk_select_noalloc(const hs2_kv_view *kv, const float *scores,
                                    int32_t *idx, int32_t idx_stride, int32_t *count,
                                    void *stream);
 
+/* Block-level variant of step 2: the granularity HySparse used and HySparse2 replaces
+ * ("HySparse2: How Xiaomi Split the Transformer to Fix Agent Prefill Costs", section "KV Reuse and
+ * Token-Level Sparse Selection": blocks of 64 tokens at the token variant's budget). For query
+ * row r at position p, with C = [0, nc), nc = max(0, p - window + 1), and W = [nc, p] as in
+ * hs2_topk_select: C is cut at multiples of block_size into blocks
+ * [j * block_size, min((j + 1) * block_size, nc)); a block's score is the float32 sum of its
+ * candidates' scores taken by folding the block in half (v[i] + v[i + n/2] for n = block_size,
+ * ..., 2, zeros past nc), a fixed order; the topk / block_size blocks with the largest score
+ * (ties: lower block index) are kept, their positions ascending, then W. If nc <= topk the
+ * selection is [0, p]. block_size: 16, 32, 64 or 128, dividing topk. The output (idx, count,
+ * idx_stride) has the layout of hs2_topk_select, so hs2_sparse_gather_attn consumes it as it
+ * is; count[r] is topk + |W| unless the chosen blocks include a short last block. workspace:
+ * device, 256-byte aligned, at least hs2_topk_select_blocks_workspace_size bytes (block scores
+ * of every row); its contents on entry do not matter. Asynchronous on `stream`; argument errors
+ * return before any launch. */
+hs2_status hs2_topk_select_blocks_workspace_size(const hs2_kv_view *kv, int32_t block_size,
+                                                 int32_t topk, int32_t window, size_t *bytes);
+hs2_status hs2_topk_select_blocks(const hs2_kv_view *kv, const float *scores,
+                                  int64_t score_stride, int32_t block_size, int32_t topk,
+                                  int32_t window, int32_t *idx, int32_t idx_stride,
+                                  int32_t *count, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
 /* Synchronises `stream` and returns the status the kernels of the last call on this workspace
  * recorded: HS2_OK, HS2_ERR_TIMEOUT or HS2_ERR_DEVICE_CHECK (HS2_ERR_CUDA if the read fails). */
 hs2_status hs2_read_device_status(const void *workspace, void *stream);

@@ -178,3 +178,26 @@ def test_selftest_rejects_bad_arguments_without_launching():
     buf = ctypes.create_string_buffer(1024)
     addr = (ctypes.addressof(buf) + 255) & ~255
     assert L.hs2_selftest_wait_timeout(0, ctypes.c_void_p(addr), 256, None) == 1   # limit 0
+
+
+def test_block_selection_argument_checks(L):
+    c = cpu_cache(lens=(300, 5000))
+    n = hs2.topk_select_blocks_workspace_size(c, 64)
+    # block scores of both rows: ceil(5000 / 64) = 79 -> stride 80 floats per row
+    assert n >= 256 + 2 * 80 * 4 and n % 256 == 0
+    for bs, topk, expect in ((48, 1024, 2), (8, 1024, 2), (256, 1024, 2), (64, 1000, 1)):
+        st = L.hs2_topk_select_blocks_workspace_size(c.ref(), bs, topk, 128,
+                                                     ctypes.byref(ctypes.c_size_t()))
+        assert st == expect, (bs, topk, L.hs2_last_error())
+    scores = torch.zeros((2, 5000))
+    idx = torch.zeros((2, 1152), dtype=torch.int32)
+    cnt = torch.zeros(2, dtype=torch.int32)
+    # too small a workspace, then too short an idx row: refused before any launch
+    st = L.hs2_topk_select_blocks(c.ref(), scores.data_ptr(), 5000, 64, 1024, 128,
+                                  idx.data_ptr(), 1152, cnt.data_ptr(), ctypes.c_void_p(256),
+                                  256, None)
+    assert st == 3 and b"workspace" in L.hs2_last_error()
+    st = L.hs2_topk_select_blocks(c.ref(), scores.data_ptr(), 5000, 64, 1024, 128,
+                                  idx.data_ptr(), 1000, cnt.data_ptr(), ctypes.c_void_p(256),
+                                  1 << 20, None)
+    assert st == 1 and b"idx_stride" in L.hs2_last_error()

@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.hs2_block_decode_traced.argtypes = [V, P, P, I32, I32, I32, F, P, P, I32, P, P, I64, P,
                                               I32, P, P, SZ, P, I32, P]
         L.hs2_topk_select_noalloc.argtypes = [V, P, I64, I32, I32, P, I32, P, P]
+        L.hs2_topk_select_blocks_workspace_size.argtypes = [V, I32, I32, I32, ctypes.POINTER(SZ)]
+        L.hs2_topk_select_blocks.argtypes = [V, P, I64, I32, I32, I32, P, I32, P, P, SZ, P]
         L.hs2_read_device_status.argtypes = [P, P]
         L.hs2_last_error.restype = ctypes.c_char_p
         L.hs2_status_string.restype = ctypes.c_char_p
@@ -91,7 +93,8 @@ def lib() -> ctypes.CDLL:
         L.hs2_selftest_wait_timeout.restype = ctypes.c_int
         for name in ("hs2_workspace_size", "hs2_full_attn_scores", "hs2_topk_select",
                      "hs2_sparse_gather_attn", "hs2_block_decode", "hs2_block_decode_traced",
-                     "hs2_topk_select_noalloc", "hs2_read_device_status"):
+                     "hs2_topk_select_noalloc", "hs2_read_device_status",
+                     "hs2_topk_select_blocks_workspace_size", "hs2_topk_select_blocks"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -190,6 +193,25 @@ def topk_select_noalloc(cache: KvCache, scores, idx, count, topk=TOPK, window=WI
     _check(lib().hs2_topk_select_noalloc(cache.ref(), _ptr(scores), scores.stride(0), topk,
                                          window, _ptr(idx), idx.stride(0), _ptr(count),
                                          _stream(stream)))
+
+
+def topk_select_blocks_workspace_size(cache: KvCache, block_size: int = 64, topk: int = TOPK,
+                                      window: int = WINDOW) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().hs2_topk_select_blocks_workspace_size(cache.ref(), block_size, topk, window,
+                                                       ctypes.byref(n)))
+    return int(n.value)
+
+
+def topk_select_blocks(cache: KvCache, scores, idx, count, workspace, block_size: int = 64,
+                       topk=TOPK, window=WINDOW, stream=None):
+    """Block-level selection (topk / block_size whole blocks plus the window); same outputs as
+    topk_select (see hs2_topk_select_blocks in include/hs2.h)."""
+    _check(lib().hs2_topk_select_blocks(cache.ref(), _ptr(scores), scores.stride(0), block_size,
+                                        topk, window, _ptr(idx), idx.stride(0), _ptr(count),
+                                        _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)))
 
 
 def sparse_gather_attn(cache: KvCache, q, idx, count, out, workspace, scale=None, stream=None):

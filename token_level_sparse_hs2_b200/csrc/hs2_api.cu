@@ -572,6 +572,34 @@ hs2_status check_full_args(const Plan &P, const void *q, float scale, const void
   return HS2_OK;
 }
 
+// Block-level selection: the workspace holds the status word and the block scores.
+constexpr int kBlockSelSmemKeys = 32768;   // block scores per row staged in shared memory
+
+struct BlockPlan {
+  int64_t blk_stride = 0;
+  size_t off_blk = 0, total = 0;
+  int pool_ctas_per_row = 0;
+};
+
+hs2_status check_block_args(int block_size, int topk) {
+  if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128)
+    return fail(HS2_ERR_UNSUPPORTED, "block_size %d (16, 32, 64 or 128)", block_size);
+  if (topk % block_size != 0)
+    return fail(HS2_ERR_INVALID_ARG, "topk %d is not a multiple of block_size %d", topk, block_size);
+  return HS2_OK;
+}
+
+BlockPlan block_plan(const Plan &P, int block_size) {
+  BlockPlan B;
+  const int64_t positions = P.max_p + 1;
+  B.blk_stride = ((positions + block_size - 1) / block_size + 3) / 4 * 4;
+  B.off_blk = align_up(4);
+  B.total = align_up(B.off_blk + (size_t)P.n_rows * (size_t)B.blk_stride * 4);
+  const int per = block_pool_positions_per_cta();
+  B.pool_ctas_per_row = (int)((positions + per - 1) / per);
+  return B;
+}
+
 }  // namespace
 }  // namespace hs2
 
@@ -662,6 +690,68 @@ hs2_status hs2_topk_select_noalloc(const hs2_kv_view *kv, const float *scores,
   sc.cand_key = ws_at<uint32_t>(base, lay.off_cand_key);
   sc.cand_idx = ws_at<int32_t>(base, lay.off_cand_idx);
   st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, false, sc, s);
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_topk_select_blocks_workspace_size(const hs2_kv_view *kv, int32_t block_size,
+                                                 int32_t topk, int32_t window, size_t *bytes) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if ((st = check_budget(topk, window)) != HS2_OK) return st;
+  if ((st = check_block_args(block_size, topk)) != HS2_OK) return st;
+  if (!bytes) return fail(HS2_ERR_INVALID_ARG, "bytes is NULL");
+  Plan P;
+  make_plan(kv, P);
+  *bytes = block_plan(P, block_size).total;
+  return ok();
+}
+
+hs2_status hs2_topk_select_blocks(const hs2_kv_view *kv, const float *scores,
+                                  int64_t score_stride, int32_t block_size, int32_t topk,
+                                  int32_t window, int32_t *idx, int32_t idx_stride,
+                                  int32_t *count, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if ((st = check_budget(topk, window)) != HS2_OK) return st;
+  if ((st = check_block_args(block_size, topk)) != HS2_OK) return st;
+  Plan P;
+  make_plan(kv, P);
+  if (!scores) return fail(HS2_ERR_INVALID_ARG, "scores is NULL");
+  if (score_stride < P.max_p + 1)
+    return fail(HS2_ERR_INVALID_ARG, "score_stride %lld < %lld", (long long)score_stride,
+                (long long)(P.max_p + 1));
+  if ((st = check_idx(P, topk, window, idx, idx_stride, count)) != HS2_OK) return st;
+  const BlockPlan B = block_plan(P, block_size);
+  if (!workspace) return fail(HS2_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign)
+    return fail(HS2_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (workspace_bytes < B.total)
+    return fail(HS2_ERR_WORKSPACE, "workspace %zu bytes < %zu required", workspace_bytes, B.total);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  BlockSelParams bp;
+  memset(&bp, 0, sizeof bp);
+  fill_seq(kv, P, bp.seq);
+  bp.batch = P.B;
+  bp.n_q = P.n_q;
+  bp.bs = block_size;
+  bp.kb = topk / block_size;
+  bp.topk = topk;
+  bp.window = window;
+  bp.scores = scores;
+  bp.score_stride = score_stride;
+  bp.blk = ws_at<float>(workspace, B.off_blk);
+  bp.blk_stride = B.blk_stride;
+  bp.pool_ctas_per_row = B.pool_ctas_per_row;
+  bp.smem_keys = (int)std::min<int64_t>(kBlockSelSmemKeys, B.blk_stride);
+  // many rows: each CTA pools its own row (one launch, no block-score round trip); few long
+  // rows: the pooling is spread over the chip first
+  bp.fused = (P.n_rows >= kManyRows && B.blk_stride <= kBlockSelSmemKeys) ? 1 : 0;
+  bp.status = ws_at<uint32_t>(workspace, 0);
+  bp.idx = idx;
+  bp.idx_stride = idx_stride;
+  bp.count = count;
+  st = cuda_check(launch_block_select(bp, P.n_rows, s), "block selection");
   return st == HS2_OK ? ok() : st;
 }
 

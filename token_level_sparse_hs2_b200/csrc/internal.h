@@ -136,6 +136,27 @@ struct TopkParams {
   uint32_t *status;
 };
 
+// Block-level selection: pooled block scores, then one CTA per query row.
+struct BlockSelParams {
+  SeqTable seq;
+  int32_t batch, n_q;
+  int32_t bs, kb, topk, window;    // block size (16 .. 128), blocks kept = topk / bs
+  const float *scores;
+  int64_t score_stride;
+  float *blk;                      // [B*n_q, blk_stride] float32 block scores
+  int64_t blk_stride;
+  int32_t pool_ctas_per_row;       // pool grid = rows x this
+  int32_t smem_keys;               // rows with at most this many blocks select in shared memory
+  int32_t fused;                   // 1: one kernel, each CTA pools its own row (needs every
+                                   // row's blocks to fit smem_keys)
+  uint32_t *status;                // workspace status word (written 0)
+  int32_t *idx;
+  int32_t idx_stride;
+  int32_t *count;
+};
+cudaError_t launch_block_select(const BlockSelParams &p, int n_rows, cudaStream_t s);
+int block_pool_positions_per_cta();
+
 // Merge of split partials into outputs: one CTA per (group, head). Group g owns partial slots
 // [slot_begin(g), slot_begin(g) + n(g)): from seq.item_begin when by_seq, else g * n_fixed.
 // Groups with a single slot were written directly by their CTA and are skipped.
