@@ -72,6 +72,7 @@ def lib():
         L.hs2o_e4m3_rne.argtypes = [ctypes.c_float]
         L.hs2o_e4m3_rne.restype = ctypes.c_uint8
         L.hs2o_quantize_row.argtypes = [P, I32, P, P]
+        L.hs2o_kv_bridge.argtypes = [P, P, I64, I32, P]
         L.hs2o_select_blocks_f64.argtypes = [P, I64, I32, I32, I32, P]
         L.hs2o_select_blocks_f64.restype = I64
         L.hs2o_select_blocks_f32.argtypes = [P, I64, I32, I32, I32, P]
@@ -267,6 +268,19 @@ def block(w, rows=None, scale=None):
                 for l in range(w.n_sparse)]
     return dict(rows=rows, o_full=o_full, lse=lse, scores=s, idx=idx, count=count,
                 o_sparse=o_sparse)
+
+
+def kv_bridge(hidden_bits: np.ndarray, w_bits: np.ndarray):
+    """KV Bridging projections: hidden bf16 bits [m, d], w bf16 bits [256, d] (K rows 0..127,
+    V rows 128..255) -> (K [m, 128], V [m, 128]) in float64."""
+    h = np.ascontiguousarray(hidden_bits, dtype=np.uint16)
+    w = np.ascontiguousarray(w_bits, dtype=np.uint16)
+    m, d = h.shape
+    if w.shape != (256, d):
+        raise ValueError("w must be [256, d]")
+    out = np.empty((m, 256), dtype=np.float64)
+    lib().hs2o_kv_bridge(h.ctypes.data, w.ctypes.data, m, d, out.ctypes.data)
+    return out[:, :128], out[:, 128:]
 
 
 def e4m3_rne(y: float) -> int:

@@ -276,6 +276,29 @@ int hs2o_select_rows_f32(const hs2o_kv *kv, const int64_t *rows, int64_t n_rows,
   return bad ? -1 : 0;
 }
 
+/* ---------------------------------------------------------------- KV Bridging */
+
+/* The cross-decoder full layer's K and V projected from a self-decoder full layer's hidden
+ * states ("HySparse2: How Xiaomi Split the Transformer to Fix Agent Prefill Costs", section
+ * "The Self-Decoder and Cross-Decoder Split": K_j = Proj_j^K(H_i^self), V_j = Proj_j^V(H_i^self),
+ * learned projections; read here as plain linear maps, no bias). hidden: bf16 bits [m, d];
+ * w: bf16 bits [256, d], rows 0..127 the K projection, 128..255 the V projection (output
+ * feature x input feature). out: [m, 256] = hidden . w^T in double, summed in index order. */
+void hs2o_kv_bridge(const uint16_t *hidden, const uint16_t *w, int64_t m, int d, double *out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < m; ++r) {
+    double *h = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!h) continue;
+    for (int e = 0; e < d; ++e) h[e] = bf16_to_double(hidden[r * d + e]);
+    for (int c = 0; c < 256; ++c) {
+      double acc = 0.0;
+      for (int e = 0; e < d; ++e) acc += h[e] * bf16_to_double(w[(int64_t)c * d + e]);
+      out[r * 256 + c] = acc;
+    }
+    free(h);
+  }
+}
+
 /* ---------------------------------------------------------------- block-level selection */
 
 /* The block-granular selection HySparse used and HySparse2 replaces ("HySparse2: How Xiaomi

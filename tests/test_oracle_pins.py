@@ -314,3 +314,34 @@ def test_quantize_rows_scale_codes_and_error_bound(oracle_lib):
     step = np.maximum(np.abs(xf) / 8.0, 2.0 ** -9 * scale[:, None])    # 3 mantissa bits; subnormal floor
     assert np.all(err <= step * 0.5 + 1e-12)
     assert codes[5, 17] == 0xfe and np.all(codes[5, np.arange(128) != 17] == 0)
+
+
+# ------------------------------------------------------------------ KV Bridging projections
+
+def test_kv_bridge_equals_float64_matmul(oracle_lib):
+    """The projections equal a library float64 matmul of the widened bf16 inputs."""
+    rng = np.random.default_rng(21)
+    m, d = 37, 192
+    h = f32_to_bf16_bits(rng.standard_normal((m, d)).astype(np.float32))
+    w = f32_to_bf16_bits((rng.standard_normal((256, d)) / np.sqrt(d)).astype(np.float32))
+    k, v = oracle_lib.kv_bridge(h, w)
+    ref = torch.from_numpy(bf16_bits_to_f32(h).astype(np.float64)) @ \
+        torch.from_numpy(bf16_bits_to_f32(w).astype(np.float64)).T
+    assert np.allclose(k, ref[:, :128].numpy(), rtol=0, atol=1e-12)
+    assert np.allclose(v, ref[:, 128:].numpy(), rtol=0, atol=1e-12)
+
+
+def test_kv_bridge_selector_weights_copy_features(oracle_lib):
+    """One-hot weight rows pick input features: K[:, c] = h[:, 2c], V[:, c] = -h[:, c + 1]."""
+    rng = np.random.default_rng(22)
+    m, d = 5, 256
+    hf = rng.standard_normal((m, d)).astype(np.float32)
+    h = f32_to_bf16_bits(hf)
+    wf = np.zeros((256, d), dtype=np.float32)
+    for c in range(128):
+        wf[c, 2 * c] = 1.0
+        wf[128 + c, c + 1] = -1.0
+    k, v = oracle_lib.kv_bridge(h, f32_to_bf16_bits(wf))
+    hb = bf16_bits_to_f32(h).astype(np.float64)
+    assert np.array_equal(k, hb[:, 0:256:2])
+    assert np.array_equal(v, -hb[:, 1:129])
