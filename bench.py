@@ -245,6 +245,37 @@ def bench_kv_append(hs2, dev, hbm, rows=65536, iters=20):
             "bytes": nbytes, "achieved_gbs": gbs, "frac": gbs / hbm}
 
 
+def bench_kv_bridge(hs2, dev, hbm, tf_burst, tokens=32768, d_model=4096, iters=10):
+    """KV Bridging on a prefill of `tokens` prompt tokens (hidden size d_model, synthetic
+    weights): K and V rows = hidden . [W_K; W_V]^T into a bf16 cache. FLOPs 2 x tokens x d_model
+    x 256; bytes = hidden + weights read, K and V rows written."""
+    g = torch.Generator(device=dev).manual_seed(7)
+    hidden = torch.randn((1, tokens, d_model), device=dev, generator=g).to(torch.bfloat16)
+    w = (torch.randn((256, d_model), device=dev, generator=g) / d_model ** 0.5).to(torch.bfloat16)
+    k = torch.empty((tokens, 128), dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    cache = hs2.KvCache(k, v, [0], [tokens], tokens, 32)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        hs2.kv_bridge(cache, hidden, w, ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(iters):
+        hs2.kv_bridge(cache, hidden, w, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / iters * 1e3
+    flops = 2.0 * tokens * d_model * 256
+    nbytes = tokens * d_model * 2 + 256 * d_model * 2 + tokens * 2 * 256
+    tf = flops / (us / 1e6) / 1e12
+    gbs = nbytes / (us / 1e6) / 1e9
+    return {"kernel": "kv_bridge_kernel", "tokens": tokens, "d_model": d_model, "us": us,
+            "flops": flops, "tflops": tf, "frac_of_bf16_burst_peak": tf / tf_burst,
+            "bytes": nbytes, "achieved_gbs": gbs, "frac_of_hbm": gbs / hbm,
+            "note": "hidden states (%.0f MB) exceed L2; no flush" % (tokens * d_model * 2 / 1e6)}
+
+
 def bench_block_select(hs2, cache, scores, w, dev, token_ms, block_size=64, iters=20):
     """Block-level selection (HySparse's granularity at the same budget) on the step's own
     scores, beside the token-level selection's traced time: pooling + per-row select."""
@@ -465,6 +496,7 @@ def main():
     if e2e:
         line["e2e"] = e2e
     line["kv_append"] = bench_kv_append(hs2, dev, hbm)
+    line["kv_bridge"] = bench_kv_bridge(hs2, dev, hbm, tf_burst)
     line["block_select"] = bench_block_select(hs2, cache, scores, w, dev, per["topk"])
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)

@@ -227,6 +227,22 @@ int32_t hs2_version(void);
  * return before any launch. */
 hs2_status hs2_kv_append(const hs2_kv_view *kv, const void *new_k, const void *new_v, void *stream);
 
+/* KV Bridging ("HySparse2: How Xiaomi Split the Transformer to Fix Agent Prefill Costs", section
+ * "The Self-Decoder and Cross-Decoder Split": the cross-decoder full layer's cache is built from a
+ * self-decoder full layer's hidden states, K_j = Proj_j^K(H_i^self), V_j = Proj_j^V(H_i^self);
+ * the projections are taken as linear maps without bias). For the n_q last tokens of every
+ * sequence (the rows hs2_kv_append writes):
+ *   K = hidden . W_K^T,  V = hidden . W_V^T   (bf16 inputs, float32 accumulation on the tensor
+ *   cores), rounded to bf16 and written to cache row kv_start[b] + kv_len[b] - n_q + i: as bf16,
+ *   or, for an e4m3 cache, quantised from that bf16 row exactly as hs2_kv_append does.
+ * hidden: device bf16 [batch, n_q, d_model], 16-byte aligned. w_kv: device bf16 [256, d_model],
+ * rows 0..127 W_K and rows 128..255 W_V (output feature x input feature), 16-byte aligned.
+ * d_model: a multiple of 64 in [64, 32768]. workspace: device, 256-byte aligned, >= 256 bytes
+ * (the status word hs2_read_device_status reads). The view's K/V (and scale) buffers are
+ * written. Asynchronous on `stream`; argument errors return before any launch. */
+hs2_status hs2_kv_bridge(const hs2_kv_view *kv, const void *hidden, int32_t d_model,
+                         const void *w_kv, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Exercises the bounded waits of the kernels: one thread waits on an mbarrier that nothing
  * arrives at, gives up after limit_us microseconds (1 .. 2e6) and records HS2_ERR_TIMEOUT in the
  * status word at the start of `workspace` (device, 256-byte aligned, >= 256 bytes), which the

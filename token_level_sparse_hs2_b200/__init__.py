@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.hs2_launch_count.restype = ctypes.c_uint64
         L.hs2_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P, SZ, P]
         L.hs2_kv_append.argtypes = [V, P, P, P]
+        L.hs2_kv_bridge.argtypes = [V, P, I32, P, P, SZ, P]
+        L.hs2_kv_bridge.restype = ctypes.c_int
         L.hs2_kv_append.restype = ctypes.c_int
         L.hs2_selftest_wait_timeout.restype = ctypes.c_int
         for name in ("hs2_workspace_size", "hs2_full_attn_scores", "hs2_topk_select",
@@ -283,3 +285,17 @@ def kv_append(cache: KvCache, new_k, new_v, stream=None):
     """Writes the n_q new tokens of every sequence (bf16 [batch, n_q, 128] each) into the last
     n_q rows of each sequence of the cache (e4m3 caches: quantised with per-row scales)."""
     _check(lib().hs2_kv_append(cache.ref(), _ptr(new_k), _ptr(new_v), _stream(stream)))
+
+
+def kv_bridge(cache: KvCache, hidden, w_kv, workspace, stream=None):
+    """KV Bridging: cache rows of each sequence's last n_q tokens = hidden . [W_K; W_V]^T
+    (hidden bf16 [batch, n_q, d_model], w_kv bf16 [256, d_model]); see hs2_kv_bridge."""
+    if hidden.dtype != torch.bfloat16 or w_kv.dtype != torch.bfloat16:
+        raise TypeError("hidden and w_kv must be bfloat16")
+    if not (hidden.is_contiguous() and w_kv.is_contiguous()):
+        raise ValueError("hidden and w_kv must be contiguous")
+    d_model = int(hidden.shape[-1])
+    if hidden.numel() != cache.n_rows * d_model or tuple(w_kv.shape) != (256, d_model):
+        raise ValueError("hidden must be [batch, n_q, d_model] and w_kv [256, d_model]")
+    _check(lib().hs2_kv_bridge(cache.ref(), _ptr(hidden), d_model, _ptr(w_kv), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)))

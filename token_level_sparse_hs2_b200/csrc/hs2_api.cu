@@ -252,6 +252,29 @@ hs2_status encode_maps(const hs2_kv_view *kv, TensorMaps &tm) {
   return HS2_OK;
 }
 
+hs2_status encode_bridge_maps(const void *hidden, int64_t m, int d_model, const void *w,
+                              BridgeMaps &tm) {
+  hs2_status st = get_encoder();
+  if (st != HS2_OK) return st;
+  memset(&tm, 0, sizeof tm);
+  const cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t strides[1] = {(cuuint64_t)d_model * 2};
+  const cuuint64_t hdims[2] = {(cuuint64_t)d_model, (cuuint64_t)m};
+  const cuuint32_t hbox[2] = {64, 128};
+  CUresult r = g_encode(&tm.h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(hidden),
+                        hdims, strides, hbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled(hidden) = %d", (int)r);
+  const cuuint64_t wdims[2] = {(cuuint64_t)d_model, 256};
+  const cuuint32_t wbox[2] = {64, 256};
+  r = g_encode(&tm.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(w), wdims, strides,
+               wbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled(weights) = %d", (int)r);
+  return HS2_OK;
+}
+
 hs2_status cuda_check(cudaError_t e, const char *what) {
   if (e != cudaSuccess) return fail(HS2_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return HS2_OK;
@@ -913,6 +936,49 @@ hs2_status hs2_kv_append(const hs2_kv_view *kv, const void *new_k, const void *n
   ap.k_scale = const_cast<float *>(kv->k_scale);
   ap.v_scale = const_cast<float *>(kv->v_scale);
   st = cuda_check(hs2::launch_kv_append(ap, static_cast<cudaStream_t>(stream)), "kv append");
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_kv_bridge(const hs2_kv_view *kv, const void *hidden, int32_t d_model,
+                         const void *w_kv, void *workspace, size_t workspace_bytes, void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if (d_model < 64 || d_model > 32768 || d_model % 64 != 0)
+    return fail(HS2_ERR_UNSUPPORTED, "d_model %d (a multiple of 64 in [64, 32768])", d_model);
+  if (!hidden || !w_kv) return fail(HS2_ERR_INVALID_ARG, "hidden / w_kv is NULL");
+  if (!aligned16(hidden) || !aligned16(w_kv))
+    return fail(HS2_ERR_INVALID_ARG, "hidden / w_kv must be 16-byte aligned");
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % kAlign)
+    return fail(HS2_ERR_INVALID_ARG, "workspace must be a 256-byte aligned device buffer");
+  if (workspace_bytes < 256)
+    return fail(HS2_ERR_WORKSPACE, "workspace %zu bytes < 256 required", workspace_bytes);
+  const int64_t m = (int64_t)kv->batch * kv->n_q;
+  if (m > (int64_t)INT32_MAX - 128) return fail(HS2_ERR_UNSUPPORTED, "too many rows");
+  Plan P;
+  make_plan(kv, P);
+  BridgeMaps tm;
+  if ((st = encode_bridge_maps(hidden, m, d_model, w_kv, tm)) != HS2_OK) return st;
+  BridgeParams bp;
+  memset(&bp, 0, sizeof bp);
+  fill_seq(kv, P, bp.seq);
+  bp.batch = P.B;
+  bp.n_q = P.n_q;
+  bp.m = (int32_t)m;
+  bp.d_model = d_model;
+  bp.fp8 = kv->kv_dtype == HS2_KV_FP8_E4M3;
+  bp.k = const_cast<void *>(kv->k);
+  bp.v = const_cast<void *>(kv->v);
+  bp.k_scale = const_cast<float *>(kv->k_scale);
+  bp.v_scale = const_cast<float *>(kv->v_scale);
+  bp.status = static_cast<uint32_t *>(workspace);
+  int dev = 0, sms = 148;
+  if ((st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) != HS2_OK) return st;
+  if ((st = cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev),
+                       "SM count")) != HS2_OK) return st;
+  const int n_tiles = (int)((m + 127) / 128);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_check(cudaMemsetAsync(workspace, 0, 4, s), "status clear")) != HS2_OK) return st;
+  st = cuda_check(launch_kv_bridge(tm, bp, std::min(n_tiles, sms), s), "KV bridging");
   return st == HS2_OK ? ok() : st;
 }
 

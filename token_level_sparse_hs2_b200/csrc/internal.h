@@ -112,6 +112,20 @@ struct AppendParams {
 };
 cudaError_t launch_kv_append(const AppendParams &p, cudaStream_t s);
 
+// KV Bridging: cache rows of each sequence's last n_q tokens projected from hidden states
+// [B * n_q, d_model] by weights [256, d_model] (K rows 0..127, V rows 128..255).
+struct BridgeParams {
+  SeqTable seq;
+  int32_t batch, n_q, m, d_model, fp8;
+  void *k, *v;                // cache rows (bf16 or e4m3)
+  float *k_scale, *v_scale;   // e4m3: per-row scales
+  uint32_t *status;
+};
+struct BridgeMaps {
+  CUtensorMap h, w;           // hidden [m, d_model], weights [256, d_model]; 64-wide boxes
+};
+cudaError_t launch_kv_bridge(const BridgeMaps &tm, const BridgeParams &p, int grid, cudaStream_t s);
+
 // Largest thread-block cluster the sparse layer may use for this cache type and head count.
 int sparse_max_cluster(int kv_dtype, int n_heads);
 

@@ -12,10 +12,9 @@
 // largest magnitude (half-warp max), scale = amax / 448 in float32 (1 for a zero row), codes =
 // cvt.rn.satfinite of the float32 product x * (1 / scale), the reciprocal correctly rounded
 // (round to nearest even, saturating at 448).
-#include <cuda_fp8.h>
-
 #include "common.cuh"
 #include "internal.h"
+#include "quant.cuh"
 
 namespace hs2 {
 
@@ -63,13 +62,11 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
     for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(x[k]));
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));   // within the half
-    const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const float sc = fp8_row_scale(amax);
     const float inv = __frcp_rn(sc);
     uint32_t c[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      c[k] = __nv_cvt_float2_to_fp8x2(make_float2(__fmul_rn(x[2 * k], inv), __fmul_rn(x[2 * k + 1], inv)),
-                                      __NV_SATFINITE, __NV_E4M3);
+    for (int k = 0; k < 4; ++k) c[k] = fp8_pair(x[2 * k], x[2 * k + 1], inv);
     if (act) {
       uint8_t *dst = reinterpret_cast<uint8_t *>(kv ? P.v : P.k) + row * kHeadDim + 8 * hl;
       *reinterpret_cast<uint2 *>(dst) = make_uint2((c[0] & 0xffffu) | (c[1] << 16), (c[2] & 0xffffu) | (c[3] << 16));
