@@ -287,6 +287,12 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, 1)
   WarpSoftmax st;
   st.init();
   griddep_wait();
+  // the workspace's zero-initialised region (status word, histograms, selection counters):
+  // every earlier kernel of the stream has finished, and the score pass and the selection
+  // read it only after this kernel has
+  for (int t = blockIdx.x * (C::kConsumers * 32) + threadIdx.x; t < P.zero_n16;
+       t += gridDim.x * (C::kConsumers * 32))
+    P.zero[t] = make_uint4(0, 0, 0, 0);
   // every warp follows all steps of the CTA so that it flushes a partial for every sequence the
   // CTA touches, and computes only on its group's steps
   for (int it = 0; it < wk.n; ++it) {

@@ -122,8 +122,15 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
     fence_barrier_init();
   }
   __syncthreads();
-  griddep_launch_dependents();
-  griddep_wait();   // idx / count come from the selection kernel
+  // idx / count come from the selection kernel. When it ran two or more launches earlier
+  // (idx_ready: sparse layers after the first), the index staging and the first gathers are
+  // issued before the wait for the previous layer, overlapping its tail. Every layer lets the
+  // next one start only after its own wait has returned, so by then the selection kernel has
+  // finished.
+  if (!P.idx_ready) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
   const int e_begin = ts * P.split_len;
   // the split's first kPreTiles tiles of row indices, staged in shared memory (coalesced)
   const int32_t *idx = P.idx + (size_t)r * P.idx_stride;
@@ -145,6 +152,10 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
   for (int it = 0; it < min(n_tiles, C::kStages); ++it)
     gather_rows<KV, HG>(P, seq_row0, p, e_begin + it * kTile, cnt, warp, stages + it * C::kStageBytes,
                         smem_u32(&full[it]), pos_of(it), bad);
+  if (P.idx_ready) {
+    griddep_wait();   // the queries may come from the previous layer
+    griddep_launch_dependents();
+  }
 
   const int hg = warp % HG, tg = warp / HG;
   const int tok0 = tg * 16;

@@ -375,7 +375,8 @@ hs2_status sm_count(int *out) {
 hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, const void *q,
                     float scale, void *out, int out_f32, float *lse, float *scores,
                     int64_t score_stride, int window, bool with_hist, void *ws,
-                    cudaStream_t stream, const std::function<hs2_status()> *mark = nullptr) {
+                    cudaStream_t stream, const std::function<hs2_status()> *mark = nullptr,
+                    bool clear_in_pass1 = false) {
   if (P.n_q != 1) {
     RowsParams rp;
     memset(&rp, 0, sizeof rp);
@@ -458,6 +459,10 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   dp.hist = with_hist ? ws_at<uint32_t>(ws, P.off_hist) : nullptr;
   dp.part = ws_at<float>(ws, P.off_part_p1);
   dp.status = ws_at<uint32_t>(ws, P.off_status);
+  if (clear_in_pass1) {   // the caller skipped the workspace clear: pass 1 does it
+    dp.zero = ws_at<uint4>(ws, 0);
+    dp.zero_n16 = (int32_t)(P.zero_end / 16);
+  }
   st = cuda_check(launch_decode_pass(0, P.kv_dtype, tm, dp, stream), "full-attention pass 1");
   if (st != HS2_OK) return st;
   if (mark && (st = (*mark)()) != HS2_OK) return st;
@@ -530,7 +535,7 @@ hs2_status run_topk(const hs2_kv_view *kv, const Plan &P, const float *scores,
 
 hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const int32_t *idx,
                       int idx_stride, const int32_t *count, float scale, void *out, int out_f32,
-                      void *ws, cudaStream_t stream) {
+                      void *ws, cudaStream_t stream, bool idx_ready = false) {
   SparseParams sp;
   memset(&sp, 0, sizeof sp);
   fill_seq(kv, P, sp.seq);
@@ -550,6 +555,7 @@ hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const
   sp.split_len = tiles_per * kTile;
   sp.n_tsplit = (int)((cap + sp.split_len - 1) / sp.split_len);
   sp.scale_log2 = scale * 1.4426950408889634f;
+  sp.idx_ready = idx_ready ? 1 : 0;
   sp.q = q;
   sp.idx = idx;
   sp.idx_stride = idx_stride;
@@ -841,19 +847,25 @@ static hs2_status block_impl(const hs2_kv_view *kv, const void *q_full,
     return cuda_check(cudaEventRecord(static_cast<cudaEvent_t>(events[ev++]), s), "event record");
   };
   if ((st = mark()) != HS2_OK) return st;
-  if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
+  // decode: the full layer's first kernel clears the workspace region itself (no separate
+  // memset node between the previous call's last kernel and this call's first)
+  const bool clear_in_pass1 = P.n_q == 1;
+  if (!clear_in_pass1 &&
+      (st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK)
+    return st;
   if ((st = mark()) != HS2_OK) return st;
   const bool hist = P.n_seg > 1;
   st = run_full(kv, P, tm, q_full, softmax_scale, out_full, out_dtype == HS2_OUT_F32, lse, scores,
-                score_stride, window, hist, workspace, s, events ? &mark : nullptr);
+                score_stride, window, hist, workspace, s, events ? &mark : nullptr, clear_in_pass1);
   if (st != HS2_OK) return st;
   st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, hist,
                 topk_scratch(P, workspace), s);
   if (st != HS2_OK) return st;
   if ((st = mark()) != HS2_OK) return st;
   for (int l = 0; l < n_sparse; ++l) {
+    // layers after the first: the selection finished before the previous layer started
     st = run_sparse(kv, P, q_sparse[l], idx, idx_stride, count, softmax_scale, out_sparse[l],
-                    out_dtype == HS2_OUT_F32, workspace, s);
+                    out_dtype == HS2_OUT_F32, workspace, s, l > 0);
     if (st != HS2_OK) return st;
     if ((st = mark()) != HS2_OK) return st;
   }

@@ -59,6 +59,8 @@ struct DecodeParams {
   uint32_t *hist;           // pass 2: [B, kHistBins] counts of candidate top digits, or null
   float *part;              // pass 1: [slots, H, kPartRow] partials
   uint32_t *status;
+  uint4 *zero;              // pass 1: clears zero_n16 16-byte words here (the workspace's
+  int32_t zero_n16;         // zero-initialised region) once the previous kernel has finished
 };
 
 // Chunk / prefill (n_q > 1). Pass 1: blocks of 128 (query, head) rows (128 / H queries);
@@ -100,6 +102,7 @@ struct SparseParams {
   void *out;
   int32_t out_f32;
   uint32_t *status;
+  int32_t idx_ready;        // idx / count were complete before the previous kernel started
 };
 
 // Cache append of n_q new rows per sequence (the last n_q rows of each sequence).

@@ -24,6 +24,8 @@ constexpr int kAppendRowsPerWarp = 8;   // two rows (one per half warp) per step
 
 // Half warp h of a warp handles one (row, matrix) per step: 8 bf16 values per lane (16 bytes).
 __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams P) {
+  griddep_launch_dependents();
+  griddep_wait();   // earlier kernels of the stream may still read the cache rows written here
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int half = lane >> 4, hl = lane & 15;
   const int n_rows = P.batch * P.n_q, n_items = 2 * n_rows;   // (matrix, row) pairs
