@@ -77,7 +77,8 @@ struct Plan {
   // workspace (byte offsets); [0, zero_end) is cleared at the start of every call
   size_t off_status = 0, off_cnt_rows = 0, off_hist = 0, off_cand_count = 0, off_arrive = 0,
          zero_end = 0;
-  size_t off_part_p1 = 0, off_part_rows = 0, off_cand_key = 0, off_cand_idx = 0, total = 0;
+  size_t off_part_p1 = 0, off_part_rows = 0, off_cand_key = 0, off_cand_idx = 0,
+         off_seg_info = 0, total = 0;
 };
 
 hs2_status validate_view(const hs2_kv_view *kv) {
@@ -175,6 +176,7 @@ void make_plan(const hs2_kv_view *kv, Plan &P) {
   const size_t cand = (P.n_seg > 1) ? (size_t)P.n_rows * kCandCapGlobal * 4 : 0;
   P.off_cand_key = o; o = align_up(o + cand);
   P.off_cand_idx = o; o = align_up(o + cand);
+  P.off_seg_info = o; o = align_up(o + (P.n_seg > 1 ? (size_t)P.n_rows * P.n_seg * 8 : 0));
   P.total = o;
 }
 
@@ -312,6 +314,7 @@ hs2_status noalloc_scratch(void **out) {
 // call, candidate buffers are not.
 struct NoallocLayout {
   size_t off_status, off_cand_count, off_arrive, off_hist, zero_end, off_cand_key, off_cand_idx,
+      off_seg_info,
       total;
 };
 
@@ -326,6 +329,7 @@ NoallocLayout noalloc_layout(const Plan &P) {
   const size_t cand = (P.n_seg > 1) ? (size_t)P.n_rows * kCandCapGlobal * 4 : 0;
   L.off_cand_key = o; o = align_up(o + cand);
   L.off_cand_idx = o; o = align_up(o + cand);
+  L.off_seg_info = o; o = align_up(o + (P.n_seg > 1 ? (size_t)P.n_rows * P.n_seg * 8 : 0));
   L.total = o;
   return L;
 }
@@ -490,6 +494,7 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
 struct TopkScratch {
   uint32_t *status = nullptr, *hist = nullptr, *cand_key = nullptr;
   int32_t *cand_idx = nullptr, *cand_count = nullptr, *arrive = nullptr;
+  int2 *seg_info = nullptr;
 };
 
 TopkScratch topk_scratch(const Plan &P, void *ws) {
@@ -500,6 +505,7 @@ TopkScratch topk_scratch(const Plan &P, void *ws) {
   t.cand_idx = ws_at<int32_t>(ws, P.off_cand_idx);
   t.cand_count = ws_at<int32_t>(ws, P.off_cand_count);
   t.arrive = ws_at<int32_t>(ws, P.off_arrive);
+  t.seg_info = ws_at<int2>(ws, P.off_seg_info);
   return t;
 }
 
@@ -524,6 +530,7 @@ hs2_status run_topk(const hs2_kv_view *kv, const Plan &P, const float *scores,
   tp.cand_key = sc.cand_key;
   tp.cand_idx = sc.cand_idx;
   tp.cand_cap = kCandCapGlobal;
+  tp.seg_info = sc.seg_info;
   tp.cand_count = sc.cand_count;
   tp.arrive = sc.arrive;
   tp.idx = idx;
@@ -718,6 +725,7 @@ hs2_status hs2_topk_select_noalloc(const hs2_kv_view *kv, const float *scores,
   sc.hist = ws_at<uint32_t>(base, lay.off_hist);
   sc.cand_key = ws_at<uint32_t>(base, lay.off_cand_key);
   sc.cand_idx = ws_at<int32_t>(base, lay.off_cand_idx);
+  sc.seg_info = ws_at<int2>(base, lay.off_seg_info);
   st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, false, sc, s);
   return st == HS2_OK ? ok() : st;
 }

@@ -145,6 +145,7 @@ struct TopkParams {
   uint32_t *cand_key;       // [B*n_q, cand_cap] (n_seg > 1)
   int32_t *cand_idx;
   int32_t cand_cap;
+  int2 *seg_info;           // [B*n_q, n_seg] (first slot, count) of each segment's run
   int32_t *cand_count;      // [B*n_q] (self-resetting)
   int32_t *arrive;          // [B*n_q] (self-resetting)
   int32_t *idx;

@@ -11,12 +11,14 @@
 // selection is an exact radix select on 32-bit keys:
 //  1. top digit (bits 31..21) histogram: from the score pass (decode) or built here;
 //  2. the bucket B1 holding the topk-th largest key; every candidate with digit >= B1 is
-//     compacted (key, index) -- typically topk plus a few hundred;
+//     compacted (key, index) in position order (a ballot per warp and step and one block-wide
+//     scan) -- typically topk plus a few hundred;
 //  3. in shared memory: the exact threshold key tau (digits 20..10, 9..0), how many keys equal
-//     to tau are taken (the lowest indices: a radix select on the index), then the selected
-//     indices are sorted (bitonic) and the window is appended.
-// Long rows are split over several CTAs (segments) that compact into a global buffer; the last
-// segment to arrive finishes the row. If the compacted set does not fit (many equal scores),
+//     to tau are taken (the lowest indices: a radix select on the index); one more ordered
+//     compaction keeps the selected candidates in ascending order, and the window is appended.
+// Long rows are split over several CTAs (segments) that compact into a global buffer and record
+// where their run starts; the last segment to arrive lays the runs out in segment order and
+// finishes the row. If the compacted set does not fit (many equal scores),
 // the finishing CTA falls back to exact digit passes and an ordered scan over the whole row.
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -37,10 +39,10 @@ struct TkSmem {
   uint32_t hist[kHistBins];
   uint32_t key[kCandCap];
   int32_t idx[kCandCap];
-  alignas(16) int32_t sel[HS2_MAX_TOPK];
+  int32_t scan[kThreadsTk];        // per (step, warp) counts of an ordered compaction
+  int32_t seg_pre[kThreadsTk + 1]; // finishing CTA: candidates before each segment
+  int32_t seg_src[kThreadsTk];     // finishing CTA: where each segment's candidates start
   int32_t warp_sums[kWarpsTk];
-  int32_t n_cand;
-  int32_t n_sel;
   int32_t bucket;
   uint32_t above;
   int32_t last;
@@ -112,31 +114,41 @@ __device__ __forceinline__ uint32_t load_key(const float *s, int64_t t) {
   return __float_as_uint(__ldg(s + t));
 }
 
-// Warp-aggregated append of (key, t) into a buffer of capacity cap; returns nothing, the
-// counter keeps counting past cap so overflow is detectable.
-template <bool kShared>
-__device__ __forceinline__ void append(bool take, uint32_t key, int32_t t, int32_t *counter,
-                                       uint32_t *kbuf, int32_t *ibuf, int cap) {
-  const unsigned m = __ballot_sync(0xffffffffu, take);
-  if (m == 0) return;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(m) - 1;
-  int base = 0;
-  if (lane == leader) base = atomicAdd(counter, __popc(m));
-  base = __shfl_sync(0xffffffffu, base, leader);
-  if (take) {
-    const int slot = base + __popc(m & ((1u << lane) - 1u));
-    if (slot < cap) {
-      kbuf[slot] = key;
-      ibuf[slot] = t;
-    }
+// Ordered compaction of one step of U elements per thread, element u of thread x standing at
+// position u * kThreadsTk + x of the step (so consecutive threads read consecutive keys): the
+// taken elements are numbered in that order, continuing from *run (the same in every thread),
+// and emit(slot, u) is called for each. A ballot per (u, warp) and one block-wide scan over the
+// U x kWarpsTk counts give every element its slot.
+template <int U, class Emit>
+__device__ __forceinline__ void ordered_append(uint32_t take_bits, TkSmem &sm, int &run, Emit emit) {
+  static_assert(U * kWarpsTk <= kThreadsTk, "one scan entry per thread");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned m[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) m[u] = __ballot_sync(0xffffffffu, (take_bits >> u) & 1u);
+  if (lane == 0) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) sm.scan[u * kWarpsTk + warp] = __popc(m[u]);
   }
+  __syncthreads();
+  const int v = threadIdx.x < U * kWarpsTk ? sm.scan[threadIdx.x] : 0;
+  int tot;
+  const int ex = block_excl_scan(v, sm.warp_sums, &tot);
+  if (threadIdx.x < U * kWarpsTk) sm.scan[threadIdx.x] = ex;
+  __syncthreads();
+  const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+    if ((take_bits >> u) & 1u) emit(run + sm.scan[u * kWarpsTk + warp] + __popc(m[u] & below), u);
+  run += tot;
+  __syncthreads();   // sm.scan is reused by the next step
 }
 
-// Exact finish on n <= kCandCap candidates in shared memory that contain every candidate with
-// top digit >= B1 (above = how many have top digit > B1). Writes the ascending selection.
+// Exact finish on n <= kCandCap candidates in shared memory, in ascending position order, that
+// contain every candidate with top digit >= B1 (above = how many have top digit > B1). Writes
+// the ascending selection.
 __device__ void finish_from_smem(TkSmem &sm, int n, int B1, uint32_t above, int topk,
-                                 int max_idx, int32_t *out) {
+                                 int32_t *out) {
   uint32_t prefix = (uint32_t)B1 << 21, mask = 0xffe00000u;
   uint32_t need = topk - above;
   const int shifts[2] = {10, 0};
@@ -183,68 +195,25 @@ __device__ void finish_from_smem(TkSmem &sm, int n, int B1, uint32_t above, int 
     }
     ithr = (int32_t)iprefix;
   }
-  // gather the selected indices
-  if (threadIdx.x == 0) sm.n_sel = 0;
-  __syncthreads();
-  for (int t = threadIdx.x; t < ((n + 31) & ~31); t += kThreadsTk) {
-    bool take = false;
-    uint32_t k = 0;
-    int32_t ix = 0;
-    if (t < n) {
-      k = sm.key[t];
-      ix = sm.idx[t];
-      take = k > tau || (k == tau && ix <= ithr);
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    if (m) {
-      const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
-      int base = 0;
-      if (lane == leader) base = atomicAdd(&sm.n_sel, __popc(m));
-      base = __shfl_sync(0xffffffffu, base, leader);
-      if (take) {
-        const int slot = base + __popc(m & ((1u << lane) - 1u));
-        if (slot < HS2_MAX_TOPK) sm.sel[slot] = ix;
-      }
+  // the candidates are in ascending position order: keep those above the threshold in that
+  // order (16 steps of kThreadsTk cover kCandCap)
+  static_assert(kCandCap == 16 * kThreadsTk, "one ordered step covers the candidates");
+  uint32_t take = 0;
+  int32_t ix[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int j = u * kThreadsTk + threadIdx.x;
+    ix[u] = 0;
+    if (j < n) {
+      const uint32_t k = sm.key[j];
+      ix[u] = sm.idx[j];
+      if (k > tau || (k == tau && ix[u] <= ithr)) take |= 1u << u;
     }
   }
-  __syncthreads();
-  // Ascending order without a full sort: bucket the kept indices by their top bits (at most
-  // 1024 buckets), place each bucket by an exclusive scan of the bucket counts, and rank each
-  // index inside its bucket by counting the smaller members (indices are distinct).
-  {
-    uint32_t *bcnt = sm.hist, *bbeg = sm.hist + 1024;
-    int32_t *tmp = reinterpret_cast<int32_t *>(sm.key);
-    const int nbits = 32 - __clz(max(1, max_idx));
-    const int shift = max(0, nbits - 10);
-    for (int t = threadIdx.x; t < 1024; t += kThreadsTk) bcnt[t] = 0;
-    __syncthreads();
-    for (int t = threadIdx.x; t < topk; t += kThreadsTk) atomicAdd(&bcnt[sm.sel[t] >> shift], 1u);
-    __syncthreads();
-    {
-      const int e0 = 2 * threadIdx.x;
-      const int loc = (int)(bcnt[e0] + bcnt[e0 + 1]);
-      int tot;
-      const int pre = block_excl_scan(loc, sm.warp_sums, &tot);
-      bbeg[e0] = pre;
-      bbeg[e0 + 1] = pre + bcnt[e0];
-    }
-    __syncthreads();
-    for (int t = threadIdx.x; t < 1024; t += kThreadsTk) bcnt[t] = 0;   // reused as fill counters
-    __syncthreads();
-    for (int t = threadIdx.x; t < topk; t += kThreadsTk) {
-      const int x = sm.sel[t], bk = x >> shift;
-      tmp[bbeg[bk] + atomicAdd(&bcnt[bk], 1u)] = x;
-    }
-    __syncthreads();
-    for (int t = threadIdx.x; t < topk; t += kThreadsTk) {
-      const int x = tmp[t], bk = x >> shift;
-      const int j0 = bbeg[bk], j1 = j0 + (int)bcnt[bk];
-      int r = j0;
-      for (int j = j0; j < j1; ++j) r += tmp[j] < x;
-      out[r] = x;
-    }
-    __syncthreads();
-  }
+  int run = 0;
+  ordered_append<16>(take, sm, run, [&](int slot, int u) {
+    if (slot < topk) out[slot] = ix[u];
+  });
 }
 
 // Exact fallback over the whole candidate row in global memory (any number of equal keys):
@@ -381,56 +350,64 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
         if (base + u * kThreadsTk + threadIdx.x < nc) atomicAdd(&sm.hist[k[u] >> 21], 1u);
     }
   }
-  if (threadIdx.x == 0) sm.n_cand = 0;
   __syncthreads();
   // 2. bucket of the topk-th largest key
   find_bucket_block(sm.hist, kHistBins, (uint32_t)P.topk, true, sm.warp_sums, &sm.bucket, &sm.above);
   const int B1 = sm.bucket;
   const uint32_t above = sm.above;
-  // 3. compact every candidate of this segment with top digit >= B1
+  // 3. compact, in position order, every candidate of this segment with top digit >= B1 (the
+  // count keeps counting past the shared-memory capacity, which selects the exact fallback)
   int32_t *gcount = P.cand_count + r;
   uint32_t *gkey = P.cand_key + (size_t)r * P.cand_cap;
   int32_t *gidx = P.cand_idx + (size_t)r * P.cand_cap;
+  int n_local = 0;
   if (in_regs) {
+    uint32_t take = 0;
 #pragma unroll
     for (int u = 0; u < kRegKeys; ++u) {
       const int64_t t = s0 + u * kThreadsTk + threadIdx.x;
-      const bool take = t < s1 && (int)(rk[u] >> 21) >= B1;
-      append<true>(take, rk[u], (int32_t)t, &sm.n_cand, sm.key, sm.idx, kCandCap);
+      if (t < s1 && (int)(rk[u] >> 21) >= B1) take |= 1u << u;
     }
+    ordered_append<kRegKeys>(take, sm, n_local, [&](int slot, int u) {
+      if (slot < kCandCap) {
+        sm.key[slot] = rk[u];
+        sm.idx[slot] = (int32_t)(s0 + u * kThreadsTk + threadIdx.x);
+      }
+    });
   }
   for (int64_t base = in_regs ? s1 : s0; base < s1; base += kThreadsTk * kUnroll) {
     uint32_t k[kUnroll];
+    uint32_t take = 0;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t t = base + u * kThreadsTk + threadIdx.x;
       k[u] = t < s1 ? load_key(s, t) : 0u;
+      if (t < s1 && (int)(k[u] >> 21) >= B1) take |= 1u << u;
     }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t t = base + u * kThreadsTk + threadIdx.x;
-      const bool take = t < s1 && (int)(k[u] >> 21) >= B1;
-      append<true>(take, k[u], (int32_t)t, &sm.n_cand, sm.key, sm.idx, kCandCap);
-    }
+    ordered_append<kUnroll>(take, sm, n_local, [&](int slot, int u) {
+      if (slot < kCandCap) {
+        sm.key[slot] = k[u];
+        sm.idx[slot] = (int32_t)(base + u * kThreadsTk + threadIdx.x);
+      }
+    });
   }
-  __syncthreads();
   int n;
   if (P.n_seg == 1) {
-    n = sm.n_cand;
+    n = n_local;
   } else {
-    // publish this segment's candidates with one global reservation (the count keeps counting
-    // past the capacity, which sends the finishing CTA to the exact fallback)
-    const int nl = sm.n_cand;
-    if (threadIdx.x == 0) sm.bucket = atomicAdd(gcount, nl);
+    // publish this segment's candidates with one global reservation and record where they
+    // went, so that the finishing CTA can lay the segments out in position order
+    if (threadIdx.x == 0) sm.bucket = atomicAdd(gcount, n_local);
     __syncthreads();
     const int base = sm.bucket;
-    const int ncopy = min(nl, kCandCap);
+    const int ncopy = min(n_local, kCandCap);
     for (int t = threadIdx.x; t < ncopy; t += kThreadsTk) {
       if (base + t < P.cand_cap) {
         gkey[base + t] = sm.key[t];
         gidx[base + t] = sm.idx[t];
       }
     }
+    if (threadIdx.x == 0) P.seg_info[(size_t)r * P.n_seg + sg] = make_int2(base, n_local);
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -441,10 +418,27 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
     if (!sm.last) return;
     __threadfence();
     n = __ldcg(gcount);
-    if (n <= kCandCap) {
-      for (int t = threadIdx.x; t < n; t += kThreadsTk) {
-        sm.key[t] = __ldcg(gkey + t);
-        sm.idx[t] = __ldcg(gidx + t);
+    if (n <= kCandCap && n <= P.cand_cap) {
+      const int ns = P.n_seg;
+      int2 info = make_int2(0, 0);
+      if (threadIdx.x < ns) info = __ldcg(&P.seg_info[(size_t)r * ns + threadIdx.x]);
+      int tot;
+      const int pre = block_excl_scan(info.y, sm.warp_sums, &tot);
+      if (threadIdx.x < ns) {
+        sm.seg_pre[threadIdx.x] = pre;
+        sm.seg_src[threadIdx.x] = info.x;
+      }
+      __syncthreads();
+      for (int j = threadIdx.x; j < n; j += kThreadsTk) {
+        int lo = 0, hi = ns - 1;   // the last segment starting at or before j
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (sm.seg_pre[mid] <= j) lo = mid;
+          else hi = mid - 1;
+        }
+        const int src = sm.seg_src[lo] + (j - sm.seg_pre[lo]);
+        sm.key[j] = __ldcg(gkey + src);
+        sm.idx[j] = __ldcg(gidx + src);
       }
     }
     __syncthreads();
@@ -455,7 +449,7 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
   }
   // 4. finish
   const bool fits = (P.n_seg == 1) ? (n <= kCandCap) : (n <= kCandCap && n <= P.cand_cap);
-  if (fits) finish_from_smem(sm, n, B1, above, P.topk, (int)(nc - 1), out);
+  if (fits) finish_from_smem(sm, n, B1, above, P.topk, out);
   else finish_from_global(sm, s, nc, B1, above, P.topk, out);
   // 5. the forced window
   for (int64_t t = nc + threadIdx.x; t <= p; t += kThreadsTk) out[P.topk + (t - nc)] = (int32_t)t;
