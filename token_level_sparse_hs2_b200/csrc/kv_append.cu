@@ -7,8 +7,8 @@
 // and Token-Level Sparse Selection": the sparse layers and the forced window read the full
 // layer's cache, so every decode step appends its token there first.
 //
-// Each warp takes 8 (row, matrix) items, one per half warp per step, every load issued before
-// any store: 128 bf16 values per row, 8 per lane. bf16 cache: a copy. e4m3 cache: the row's
+// Each warp takes 16 (row, matrix) items, one per quarter warp per step, every load issued
+// before any store: 128 bf16 values per row, 32 per lane. bf16 cache: a copy. e4m3 cache: the row's
 // largest magnitude (half-warp max), scale = amax / 448 in float32 (1 for a zero row), codes =
 // cvt.rn.satfinite of the float32 product x * (1 / scale), the reciprocal correctly rounded
 // (round to nearest even, saturating at 448).
@@ -20,59 +20,88 @@ namespace hs2 {
 
 namespace {
 
-constexpr int kAppendRowsPerWarp = 8;   // two rows (one per half warp) per step, four steps
+constexpr int kLanesPerRow = 4;                        // 32 values (64 bytes of bf16) per lane
+constexpr int kItemsPerStep = 32 / kLanesPerRow;       // (matrix, row) items per warp step
+constexpr int kSteps = 2;                              // steps per warp, loads of both first
 
-// Half warp h of a warp handles one (row, matrix) per step: 8 bf16 values per lane (16 bytes).
+// Quarter warp q of a warp handles one (matrix, row) item per step; lane l of the quarter holds
+// values [32 l, 32 l + 32) of the row. Every per-row scalar (the destination row, the scale and
+// its reciprocal) is computed once per 8 rows of the warp, and the row maximum takes two
+// shuffles.
 __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams P) {
   griddep_launch_dependents();
   griddep_wait();   // earlier kernels of the stream may still read the cache rows written here
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  const int half = lane >> 4, hl = lane & 15;
+  const int q = lane / kLanesPerRow, ql = lane % kLanesPerRow;
   const int n_rows = P.batch * P.n_q, n_items = 2 * n_rows;   // (matrix, row) pairs
-  uint4 raw[kAppendRowsPerWarp / 2];
-  int item[kAppendRowsPerWarp / 2];
+  uint4 raw[kSteps][4];
+  int item[kSteps];
 #pragma unroll
-  for (int u = 0; u < kAppendRowsPerWarp / 2; ++u) {   // all loads first
-    item[u] = warp * kAppendRowsPerWarp + 2 * u + half;
-    raw[u] = make_uint4(0, 0, 0, 0);
+  for (int u = 0; u < kSteps; ++u) {   // all loads first
+    item[u] = (warp * kSteps + u) * kItemsPerStep + q;
     if (item[u] < n_items) {
-      const int kv = item[u] / n_rows, r = item[u] % n_rows;
-      raw[u] = *(reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(kv ? P.new_v : P.new_k) +
-                                                (size_t)r * kHeadDim) + hl);
+      const int kv = item[u] >= n_rows, r = item[u] - (kv ? n_rows : 0);
+      const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(kv ? P.new_v : P.new_k) +
+                                                         (size_t)r * kHeadDim) + 4 * ql;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) raw[u][k] = src[k];
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) raw[u][k] = make_uint4(0, 0, 0, 0);
     }
   }
 #pragma unroll
-  for (int u = 0; u < kAppendRowsPerWarp / 2; ++u) {
+  for (int u = 0; u < kSteps; ++u) {
     const bool act = item[u] < n_items;
-    const int kv = act ? item[u] / n_rows : 0, r = act ? item[u] % n_rows : 0;
-    const int b = r / P.n_q, i = r % P.n_q;
+    const int kv = act && item[u] >= n_rows;
+    const int r = act ? item[u] - (kv ? n_rows : 0) : 0;
+    int b = r, i = 0;
+    if (P.n_q != 1) {
+      b = r / P.n_q;
+      i = r - b * P.n_q;
+    }
     const int64_t row = P.seq.start[b] + (int64_t)P.seq.len[b] - P.n_q + i;
     if (!P.fp8) {
-      if (act) *(reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(kv ? P.v : P.k) + row * (kHeadDim * 2)) + hl) = raw[u];
-      continue;
-    }
-    float x[8];
-    const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+      if (act) {
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(kv ? P.v : P.k) + row * (kHeadDim * 2)) + 4 * ql;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[k]));
-      x[2 * k] = f.x;
-      x[2 * k + 1] = f.y;
+        for (int k = 0; k < 4; ++k) dst[k] = raw[u][k];
+      }
+      continue;
     }
     float amax = 0.f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) amax = fmaxf(amax, fabsf(x[k]));
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w[4] = {raw[u][k].x, raw[u][k].y, raw[u][k].z, raw[u][k].w};
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));   // within the half
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+        amax = fmax3(amax, fabsf(f.x), fabsf(f.y));
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < kLanesPerRow; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sc = fp8_row_scale(amax);
     const float inv = __frcp_rn(sc);
-    uint32_t c[4];
+    uint4 c[2];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) c[k] = fp8_pair(x[2 * k], x[2 * k + 1], inv);
+    for (int k = 0; k < 4; ++k) {   // 8 values -> 8 codes (2 words)
+      const uint32_t w[4] = {raw[u][k].x, raw[u][k].y, raw[u][k].z, raw[u][k].w};
+      uint32_t cw[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[2 * h]));
+        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[2 * h + 1]));
+        cw[h] = (fp8_pair(f0.x, f0.y, inv) & 0xffffu) | (fp8_pair(f1.x, f1.y, inv) << 16);
+      }
+      if (k & 1) { c[k >> 1].z = cw[0]; c[k >> 1].w = cw[1]; }
+      else { c[k >> 1].x = cw[0]; c[k >> 1].y = cw[1]; }
+    }
     if (act) {
-      uint8_t *dst = reinterpret_cast<uint8_t *>(kv ? P.v : P.k) + row * kHeadDim + 8 * hl;
-      *reinterpret_cast<uint2 *>(dst) = make_uint2((c[0] & 0xffffu) | (c[1] << 16), (c[2] & 0xffffu) | (c[3] << 16));
-      if (hl == 0) (kv ? P.v_scale : P.k_scale)[row] = sc;
+      uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(kv ? P.v : P.k) + row * kHeadDim + 32 * ql);
+      dst[0] = c[0];
+      dst[1] = c[1];
+      if (ql == 0) (kv ? P.v_scale : P.k_scale)[row] = sc;
     }
   }
 }
@@ -80,7 +109,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
 }  // namespace
 
 cudaError_t launch_kv_append(const AppendParams &p, cudaStream_t s) {
-  const int warps = (2 * p.batch * p.n_q + kAppendRowsPerWarp - 1) / kAppendRowsPerWarp;
+  const int per_warp = kSteps * kItemsPerStep;
+  const int warps = (2 * p.batch * p.n_q + per_warp - 1) / per_warp;
   const int grid = (warps * 32 + 255) / 256;
   cudaError_t e = launch_pdl(kv_append_kernel, grid, 256, 0, s, p);
   if (e != cudaSuccess) return e;
