@@ -227,6 +227,81 @@ int32_t hs2_version(void);
  * return before any launch. */
 hs2_status hs2_kv_append(const hs2_kv_view *kv, const void *new_k, const void *new_v, void *stream);
 
+/* ---- Context-parallel decode: one sequence's cache split by token range over ranks ----------
+ * A rank holds rows [off, off + T_local) of a sequence whose decode query sits at global position
+ * T_global - 1, as an ordinary view of T_local rows (n_q = 1; the local query position is then
+ * its last row, and every local row precedes the query). One block step is:
+ *   1. hs2_full_attn on the shard -> (O_r, lse_r); all-gather; hs2_lse_merge -> O, lse;
+ *   2. hs2_score_pass on the shard with the merged lse -> the shard's scores (global scores of
+ *      its positions); hs2_topk_select on the shard with the local window
+ *      T_local - clamp(T_global - window - off, 0, T_local) -> its top-k;
+ *      hs2_cp_pack_candidates -> its (score, global position) keys; all-gather;
+ *      hs2_cp_merge_select -> the global selection S (the same on every rank);
+ *   3. per sparse layer: hs2_cp_localize (S -> the shard's positions in S),
+ *      hs2_sparse_gather_attn_partial -> (O_r, lse_r); all-gather; hs2_lse_merge -> O.
+ * Attention over a union of disjoint position sets is the log-sum-exp merge of the parts, the
+ * score of a position needs only the global lse, and the global top-k lies inside the union of
+ * the shards' own top-k, so the result equals one GPU's over the whole context (up to the
+ * float rounding of the merges; the selection is exact on the scores the ranks computed).
+ * "HySparse2: Hybrid Sparse Attention with Two-Level KV Sharing", bullet "Inference cost" (1M-token
+ * contexts). The collectives are the caller's (torch.distributed over NCCL). */
+
+/* Step 1 alone (decode, n_q = 1): out and lse as hs2_full_attn_scores, no scores. */
+hs2_status hs2_full_attn(const hs2_kv_view *kv, const void *q, float softmax_scale, void *out,
+                         int32_t out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/* The score pass alone (decode, n_q = 1) with a given lse (device fp32 [B, H], e.g. merged over
+ * context shards): scores[b * score_stride + t] = sum_h exp(c q_h.k_t - lse[b, h]), t < kv_len[b]. */
+hs2_status hs2_score_pass(const hs2_kv_view *kv, const void *q, float softmax_scale,
+                          const float *lse, float *scores, int64_t score_stride, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
+/* hs2_sparse_gather_attn with fp32 out and the log-sum-exp of the attended scores in lse
+ * (device fp32 [B * n_q, H]); count[r] may be 0 (out = 0, lse = -inf). */
+hs2_status hs2_sparse_gather_attn_partial(const hs2_kv_view *kv, const void *q,
+                                          const int32_t *idx, int32_t idx_stride,
+                                          const int32_t *count, float softmax_scale, float *out,
+                                          float *lse, void *workspace, size_t workspace_bytes,
+                                          void *stream);
+
+/* Log-sum-exp merge of n_parts attention results over disjoint position sets:
+ *   M = max_j lse_j, w_j = exp(lse_j - M), out = sum_j w_j out_j / sum_j w_j,
+ *   lse = M + log sum_j w_j   (parts with lse = -inf contribute nothing; all empty: 0, -inf).
+ * part_out: device fp32 [n_parts, rows, H, 128]; part_lse: device fp32 [n_parts, rows, H];
+ * out: device [rows, H, 128] of out_dtype; lse: device fp32 [rows, H] or NULL. */
+hs2_status hs2_lse_merge(int32_t n_parts, int64_t rows, int32_t n_heads, const float *part_out,
+                         const float *part_lse, void *out, int32_t out_dtype, float *lse,
+                         void *stream);
+
+/* A shard's selected candidates as keys for the global merge: for entries j < count[b] of the
+ * shard's own selection idx[b] (local positions), global position g = global_offset[b] + idx,
+ * kept if g < global_len[b] - window (a global candidate); key = (fp32 bits of the score) << 32 |
+ * (0xffffffff - g), so larger keys are higher scores, then lower positions. keys: device u64
+ * [B, topk], unused slots 0. global_offset / global_len: HOST [B]. */
+hs2_status hs2_cp_pack_candidates(const hs2_kv_view *kv, const int64_t *global_offset,
+                                  const int32_t *global_len, const float *scores,
+                                  int64_t score_stride, const int32_t *idx, int32_t idx_stride,
+                                  const int32_t *count, int32_t topk, int32_t window,
+                                  uint64_t *keys, void *stream);
+
+/* The global selection from every shard's keys (device u64 [n_parts, batch, topk], n_parts x topk
+ * <= 16384): with p = global_len[b] - 1 and nc = max(0, p - window + 1), all of [0, p] if
+ * nc <= topk, else the topk largest keys' positions ascending, then [nc, p] -- what
+ * hs2_topk_select gives on the whole context's scores. idx: device int32 [batch, idx_stride]
+ * (global positions), count: device int32 [batch]. global_len: HOST [batch]. */
+hs2_status hs2_cp_merge_select(int32_t n_parts, int32_t batch, const int32_t *global_len,
+                               const uint64_t *keys, int32_t topk, int32_t window, int32_t *idx,
+                               int32_t idx_stride, int32_t *count, void *stream);
+
+/* The shard's part of an ascending global selection: entries g in [global_offset[b],
+ * global_offset[b] + local_len[b]) as local positions g - global_offset[b], in order (a
+ * contiguous run), count_local[b] of them (possibly 0). global_offset / local_len: HOST [batch]. */
+hs2_status hs2_cp_localize(int32_t batch, const int64_t *global_offset, const int32_t *local_len,
+                           const int32_t *idx, int32_t idx_stride, const int32_t *count,
+                           int32_t *idx_local, int32_t idx_local_stride, int32_t *count_local,
+                           void *stream);
+
 /* KV Bridging ("HySparse2: How Xiaomi Split the Transformer to Fix Agent Prefill Costs", section
  * "The Self-Decoder and Cross-Decoder Split": the cross-decoder full layer's cache is built from a
  * self-decoder full layer's hidden states, K_j = Proj_j^K(H_i^self), V_j = Proj_j^V(H_i^self);

@@ -91,6 +91,17 @@ def lib() -> ctypes.CDLL:
         L.hs2_kv_append.argtypes = [V, P, P, P]
         L.hs2_kv_bridge.argtypes = [V, P, I32, P, P, SZ, P]
         L.hs2_kv_bridge.restype = ctypes.c_int
+        L.hs2_full_attn.argtypes = [V, P, F, P, I32, P, P, SZ, P]
+        L.hs2_score_pass.argtypes = [V, P, F, P, P, I64, P, SZ, P]
+        L.hs2_sparse_gather_attn_partial.argtypes = [V, P, P, I32, P, F, P, P, P, SZ, P]
+        L.hs2_lse_merge.argtypes = [I32, I64, I32, P, P, P, I32, P, P]
+        L.hs2_cp_pack_candidates.argtypes = [V, P, P, P, I64, P, I32, P, I32, I32, P, P]
+        L.hs2_cp_merge_select.argtypes = [I32, I32, P, P, I32, I32, P, I32, P, P]
+        L.hs2_cp_localize.argtypes = [I32, P, P, P, I32, P, P, I32, P, P]
+        for name in ("hs2_full_attn", "hs2_score_pass", "hs2_sparse_gather_attn_partial",
+                     "hs2_lse_merge", "hs2_cp_pack_candidates", "hs2_cp_merge_select",
+                     "hs2_cp_localize"):
+            getattr(L, name).restype = ctypes.c_int
         L.hs2_kv_append.restype = ctypes.c_int
         L.hs2_selftest_wait_timeout.restype = ctypes.c_int
         for name in ("hs2_workspace_size", "hs2_full_attn_scores", "hs2_topk_select",
@@ -299,3 +310,71 @@ def kv_bridge(cache: KvCache, hidden, w_kv, workspace, stream=None):
         raise ValueError("hidden must be [batch, n_q, d_model] and w_kv [256, d_model]")
     _check(lib().hs2_kv_bridge(cache.ref(), _ptr(hidden), d_model, _ptr(w_kv), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ---------------------------------------------------------------- context-parallel pieces
+
+def _host_i64(xs):
+    return (ctypes.c_int64 * len(xs))(*[int(x) for x in xs])
+
+
+def _host_i32(xs):
+    return (ctypes.c_int32 * len(xs))(*[int(x) for x in xs])
+
+
+def full_attn(cache: KvCache, q, out, lse, workspace, scale=None, stream=None):
+    """Full-attention output and lse only (decode), see hs2_full_attn."""
+    scale = default_scale() if scale is None else scale
+    _check(lib().hs2_full_attn(cache.ref(), _ptr(q), scale, _ptr(out), _out_dtype(out), _ptr(lse),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream)))
+
+
+def score_pass(cache: KvCache, q, lse, scores, workspace, scale=None, stream=None):
+    """Importance scores with a given lse (decode), see hs2_score_pass."""
+    scale = default_scale() if scale is None else scale
+    _check(lib().hs2_score_pass(cache.ref(), _ptr(q), scale, _ptr(lse), _ptr(scores),
+                                scores.stride(0), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def sparse_gather_attn_partial(cache: KvCache, q, idx, count, out, lse, workspace, scale=None,
+                               stream=None):
+    """A sparse layer's fp32 output and lse over the given (possibly empty) selection."""
+    scale = default_scale() if scale is None else scale
+    _check(lib().hs2_sparse_gather_attn_partial(cache.ref(), _ptr(q), _ptr(idx), idx.stride(0),
+                                                _ptr(count), scale, _ptr(out), _ptr(lse),
+                                                _ptr(workspace),
+                                                workspace.numel() * workspace.element_size(),
+                                                _stream(stream)))
+
+
+def lse_merge(part_out, part_lse, out, lse=None, stream=None):
+    """Log-sum-exp merge of [n_parts, rows, H, 128] outputs with [n_parts, rows, H] lse."""
+    if not (part_out.is_contiguous() and part_lse.is_contiguous() and out.is_contiguous()):
+        raise ValueError("lse_merge needs contiguous tensors")
+    n_parts, rows, heads = part_lse.shape[0], part_lse.shape[1], part_lse.shape[2]
+    _check(lib().hs2_lse_merge(n_parts, rows, heads, _ptr(part_out), _ptr(part_lse), _ptr(out),
+                               _out_dtype(out), _ptr(lse), _stream(stream)))
+
+
+def cp_pack_candidates(cache: KvCache, global_offset, global_len, scores, idx, count, keys,
+                       topk=TOPK, window=WINDOW, stream=None):
+    _check(lib().hs2_cp_pack_candidates(cache.ref(), _host_i64(global_offset),
+                                        _host_i32(global_len), _ptr(scores), scores.stride(0),
+                                        _ptr(idx), idx.stride(0), _ptr(count), topk, window,
+                                        _ptr(keys), _stream(stream)))
+
+
+def cp_merge_select(keys, global_len, idx, count, topk=TOPK, window=WINDOW, stream=None):
+    """keys: int64 [n_parts, batch, topk] (the u64 keys of every shard)."""
+    n_parts, batch = keys.shape[0], keys.shape[1]
+    _check(lib().hs2_cp_merge_select(n_parts, batch, _host_i32(global_len), _ptr(keys), topk,
+                                     window, _ptr(idx), idx.stride(0), _ptr(count),
+                                     _stream(stream)))
+
+
+def cp_localize(global_offset, local_len, idx, count, idx_local, count_local, stream=None):
+    _check(lib().hs2_cp_localize(len(local_len), _host_i64(global_offset), _host_i32(local_len),
+                                 _ptr(idx), idx.stride(0), _ptr(count), _ptr(idx_local),
+                                 idx_local.stride(0), _ptr(count_local), _stream(stream)))

@@ -137,9 +137,10 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
   const int n_pre = min(min(P.split_len, kPreTiles * kTile), P.idx_stride - e_begin);
   for (int t = threadIdx.x; t < n_pre; t += C::kThreads) s_idx[t] = __ldcg(idx + e_begin + t);
   int cnt = __ldcg(P.count + r);
-  if (cnt < 1 || cnt > P.idx_stride) {
+  const int cmin = P.allow_empty ? 0 : 1;
+  if (cnt < cmin || cnt > P.idx_stride) {
     if (threadIdx.x == 0) record_status(P.status, kStatusCheck);
-    cnt = max(1, min(cnt, P.idx_stride));
+    cnt = max(cmin, min(cnt, P.idx_stride));
   }
   const int n_tiles = max(0, min(P.split_len, cnt - e_begin) + kTile - 1) / kTile;
   __syncthreads();   // s_idx
@@ -278,7 +279,10 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
       O.w += o.w;
     }
     if (P.n_tsplit == 1) {
-      const float inv = 1.f / hml[2 * h + 1];
+      const float Lh = hml[2 * h + 1];
+      const float inv = Lh > 0.f ? 1.f / Lh : 0.f;   // 0: a shard that holds none of the selection
+      if (P.lse_out && d4 == 0)
+        P.lse_out[(size_t)r * H + h] = Lh > 0.f ? (hml[2 * h] + __log2f(Lh)) * kLn2 : -INFINITY;
       const size_t oi = ((size_t)r * H + h) * kHeadDim + 4 * d4;
       if (P.out_f32) {
         *reinterpret_cast<float4 *>(reinterpret_cast<float *>(P.out) + oi) =
@@ -336,7 +340,9 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
         }
       }
     }
-    const float inv = 1.f / L;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    if (P.lse_out && lane == 0)
+      P.lse_out[(size_t)r * H + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
     const size_t oi = ((size_t)r * H + h) * kHeadDim + 4 * lane;
     if (P.out_f32) {
       *reinterpret_cast<float4 *>(reinterpret_cast<float *>(P.out) + oi) =

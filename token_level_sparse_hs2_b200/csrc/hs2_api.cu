@@ -380,7 +380,7 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
                     float scale, void *out, int out_f32, float *lse, float *scores,
                     int64_t score_stride, int window, bool with_hist, void *ws,
                     cudaStream_t stream, const std::function<hs2_status()> *mark = nullptr,
-                    bool clear_in_pass1 = false) {
+                    bool clear_in_pass1 = false, int passes = 3) {
   if (P.n_q != 1) {
     RowsParams rp;
     memset(&rp, 0, sizeof rp);
@@ -467,6 +467,10 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
     dp.zero = ws_at<uint4>(ws, 0);
     dp.zero_n16 = (int32_t)(P.zero_end / 16);
   }
+  if (!(passes & 1)) {   // score pass only, with the caller's lse
+    st = cuda_check(launch_decode_pass(1, P.kv_dtype, tm, dp, stream), "score pass 2");
+    return st;
+  }
   st = cuda_check(launch_decode_pass(0, P.kv_dtype, tm, dp, stream), "full-attention pass 1");
   if (st != HS2_OK) return st;
   if (mark && (st = (*mark)()) != HS2_OK) return st;
@@ -484,6 +488,7 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
     if ((st = cuda_check(launch_merge(mp, stream), "pass 1 merge")) != HS2_OK) return st;
   }
   if (mark && (st = (*mark)()) != HS2_OK) return st;
+  if (!(passes & 2)) return HS2_OK;
   st = cuda_check(launch_decode_pass(1, P.kv_dtype, tm, dp, stream), "score pass 2");
   if (st != HS2_OK) return st;
   if (mark && (st = (*mark)()) != HS2_OK) return st;
@@ -542,7 +547,8 @@ hs2_status run_topk(const hs2_kv_view *kv, const Plan &P, const float *scores,
 
 hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const int32_t *idx,
                       int idx_stride, const int32_t *count, float scale, void *out, int out_f32,
-                      void *ws, cudaStream_t stream, bool idx_ready = false) {
+                      void *ws, cudaStream_t stream, bool idx_ready = false,
+                      float *lse_out = nullptr, bool allow_empty = false) {
   SparseParams sp;
   memset(&sp, 0, sizeof sp);
   fill_seq(kv, P, sp.seq);
@@ -563,6 +569,8 @@ hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const
   sp.n_tsplit = (int)((cap + sp.split_len - 1) / sp.split_len);
   sp.scale_log2 = scale * 1.4426950408889634f;
   sp.idx_ready = idx_ready ? 1 : 0;
+  sp.lse_out = lse_out;
+  sp.allow_empty = allow_empty ? 1 : 0;
   sp.q = q;
   sp.idx = idx;
   sp.idx_stride = idx_stride;
@@ -956,6 +964,189 @@ hs2_status hs2_kv_append(const hs2_kv_view *kv, const void *new_k, const void *n
   ap.k_scale = const_cast<float *>(kv->k_scale);
   ap.v_scale = const_cast<float *>(kv->v_scale);
   st = cuda_check(hs2::launch_kv_append(ap, static_cast<cudaStream_t>(stream)), "kv append");
+  return st == HS2_OK ? ok() : st;
+}
+
+// ------------------------------------------------------------------ context-parallel pieces
+
+hs2_status hs2_full_attn(const hs2_kv_view *kv, const void *q, float softmax_scale, void *out,
+                         int32_t out_dtype, float *lse, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if (kv->n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "hs2_full_attn is for decode (n_q = 1)");
+  Plan P;
+  make_plan(kv, P);
+  float dummy_scores = 0.f;   // not written: the score pass does not run
+  if ((st = check_full_args(P, q, softmax_scale, out, out_dtype, lse, &dummy_scores, P.max_p + 1)) != HS2_OK)
+    return st;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
+  TensorMaps tm;
+  if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = run_full(kv, P, tm, q, softmax_scale, out, out_dtype == HS2_OUT_F32, lse, nullptr, 0, 0,
+                false, workspace, s, nullptr, true, 1);
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_score_pass(const hs2_kv_view *kv, const void *q, float softmax_scale,
+                          const float *lse, float *scores, int64_t score_stride, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if (kv->n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "hs2_score_pass is for decode (n_q = 1)");
+  Plan P;
+  make_plan(kv, P);
+  int dummy_out = 0;
+  if ((st = check_full_args(P, q, softmax_scale, q, HS2_OUT_F32, lse, scores, score_stride)) != HS2_OK)
+    return st;
+  (void)dummy_out;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
+  TensorMaps tm;
+  if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
+  st = run_full(kv, P, tm, q, softmax_scale, nullptr, 0, const_cast<float *>(lse), scores,
+                score_stride, 0, false, workspace, s, nullptr, false, 2);
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_sparse_gather_attn_partial(const hs2_kv_view *kv, const void *q,
+                                          const int32_t *idx, int32_t idx_stride,
+                                          const int32_t *count, float softmax_scale, float *out,
+                                          float *lse, void *workspace, size_t workspace_bytes,
+                                          void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  Plan P;
+  make_plan(kv, P);
+  if (!q || !out || !lse) return fail(HS2_ERR_INVALID_ARG, "q / out / lse is NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(HS2_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
+  if (!idx || !count) return fail(HS2_ERR_INVALID_ARG, "idx / count is NULL");
+  if (idx_stride < 1) return fail(HS2_ERR_INVALID_ARG, "idx_stride %d < 1", idx_stride);
+  if (!valid_scale(softmax_scale)) return fail(HS2_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_check(cudaMemsetAsync(workspace, 0, P.zero_end, s), "workspace clear")) != HS2_OK) return st;
+  st = run_sparse(kv, P, q, idx, idx_stride, count, softmax_scale, out, 1, workspace, s, false,
+                  lse, true);
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_lse_merge(int32_t n_parts, int64_t rows, int32_t n_heads, const float *part_out,
+                         const float *part_lse, void *out, int32_t out_dtype, float *lse,
+                         void *stream) {
+  if (n_parts < 1 || n_parts > 1024) return fail(HS2_ERR_INVALID_ARG, "n_parts %d outside [1, 1024]", n_parts);
+  if (rows < 0 || n_heads < 1 || rows * n_heads > INT32_MAX)
+    return fail(HS2_ERR_INVALID_ARG, "rows %lld x n_heads %d out of range", (long long)rows, n_heads);
+  if (!part_out || !part_lse || !out) return fail(HS2_ERR_INVALID_ARG, "part_out / part_lse / out is NULL");
+  if (out_dtype != HS2_OUT_BF16 && out_dtype != HS2_OUT_F32)
+    return fail(HS2_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
+  LseMergeParams mp;
+  memset(&mp, 0, sizeof mp);
+  mp.n_parts = n_parts;
+  mp.n_heads = n_heads;
+  mp.rows = rows;
+  mp.part_o = part_out;
+  mp.part_lse = part_lse;
+  mp.out = out;
+  mp.out_f32 = out_dtype == HS2_OUT_F32;
+  mp.lse = lse;
+  hs2_status st = cuda_check(launch_lse_merge(mp, static_cast<cudaStream_t>(stream)), "lse merge");
+  return st == HS2_OK ? ok() : st;
+}
+
+namespace {
+hs2_status cp_fill(CpParams &cp, int32_t batch, const int64_t *offset, const int32_t *local_len,
+                   const int32_t *global_len) {
+  memset(&cp, 0, sizeof cp);
+  if (batch < 1 || batch > HS2_MAX_BATCH)
+    return fail(HS2_ERR_INVALID_ARG, "batch %d outside [1, %d]", batch, HS2_MAX_BATCH);
+  cp.batch = batch;
+  for (int b = 0; b < batch; ++b) {
+    if (offset) cp.offset[b] = offset[b];
+    if (local_len) cp.local_len[b] = local_len[b];
+    if (global_len) cp.global_len[b] = global_len[b];
+    if ((offset && offset[b] < 0) || (local_len && local_len[b] < 1) || (global_len && global_len[b] < 1))
+      return fail(HS2_ERR_INVALID_ARG, "sequence %d: bad offset or length", b);
+    if (offset && local_len && global_len && offset[b] + local_len[b] > global_len[b])
+      return fail(HS2_ERR_INVALID_ARG, "sequence %d: shard [%lld, %lld) past the context (%d)", b,
+                  (long long)offset[b], (long long)(offset[b] + local_len[b]), global_len[b]);
+  }
+  return HS2_OK;
+}
+}  // namespace
+
+hs2_status hs2_cp_pack_candidates(const hs2_kv_view *kv, const int64_t *global_offset,
+                                  const int32_t *global_len, const float *scores,
+                                  int64_t score_stride, const int32_t *idx, int32_t idx_stride,
+                                  const int32_t *count, int32_t topk, int32_t window,
+                                  uint64_t *keys, void *stream) {
+  hs2_status st = validate_view(kv);
+  if (st != HS2_OK) return st;
+  if (kv->n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "context-parallel decode needs n_q = 1");
+  if ((st = check_budget(topk, window)) != HS2_OK) return st;
+  if (!global_offset || !global_len) return fail(HS2_ERR_INVALID_ARG, "global_offset / global_len is NULL");
+  if (!scores || !idx || !count || !keys) return fail(HS2_ERR_INVALID_ARG, "scores / idx / count / keys is NULL");
+  if (idx_stride < 1 || score_stride < 1) return fail(HS2_ERR_INVALID_ARG, "bad stride");
+  CpParams cp;
+  if ((st = cp_fill(cp, kv->batch, global_offset, kv->kv_len, global_len)) != HS2_OK) return st;
+  for (int b = 0; b < kv->batch; ++b)
+    if (score_stride < kv->kv_len[b]) return fail(HS2_ERR_INVALID_ARG, "score_stride < kv_len[%d]", b);
+  cp.topk = topk;
+  cp.window = window;
+  cp.scores = scores;
+  cp.score_stride = score_stride;
+  cp.idx = idx;
+  cp.idx_stride = idx_stride;
+  cp.count = count;
+  cp.keys = keys;
+  st = cuda_check(launch_cp_pack(cp, static_cast<cudaStream_t>(stream)), "candidate pack");
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_cp_merge_select(int32_t n_parts, int32_t batch, const int32_t *global_len,
+                               const uint64_t *keys, int32_t topk, int32_t window, int32_t *idx,
+                               int32_t idx_stride, int32_t *count, void *stream) {
+  hs2_status st = check_budget(topk, window);
+  if (st != HS2_OK) return st;
+  if (n_parts < 1 || (int64_t)n_parts * topk > kCpMaxKeys)
+    return fail(HS2_ERR_UNSUPPORTED, "n_parts %d x topk %d above %d", n_parts, topk, kCpMaxKeys);
+  if (!global_len || !keys || !idx || !count) return fail(HS2_ERR_INVALID_ARG, "NULL argument");
+  CpParams cp;
+  if ((st = cp_fill(cp, batch, nullptr, nullptr, global_len)) != HS2_OK) return st;
+  for (int b = 0; b < batch; ++b)
+    if (idx_stride < std::min<int64_t>(global_len[b], (int64_t)topk + window))
+      return fail(HS2_ERR_INVALID_ARG, "idx_stride %d too small for sequence %d", idx_stride, b);
+  cp.n_parts = n_parts;
+  cp.topk = topk;
+  cp.window = window;
+  cp.keys = const_cast<uint64_t *>(keys);
+  cp.idx_out = idx;
+  cp.out_stride = idx_stride;
+  cp.count_out = count;
+  st = cuda_check(launch_cp_select(cp, static_cast<cudaStream_t>(stream)), "candidate merge");
+  return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_cp_localize(int32_t batch, const int64_t *global_offset, const int32_t *local_len,
+                           const int32_t *idx, int32_t idx_stride, const int32_t *count,
+                           int32_t *idx_local, int32_t idx_local_stride, int32_t *count_local,
+                           void *stream) {
+  if (!global_offset || !local_len || !idx || !count || !idx_local || !count_local)
+    return fail(HS2_ERR_INVALID_ARG, "NULL argument");
+  if (idx_stride < 1 || idx_local_stride < idx_stride)
+    return fail(HS2_ERR_INVALID_ARG, "idx_local_stride %d < idx_stride %d", idx_local_stride, idx_stride);
+  CpParams cp;
+  hs2_status st = cp_fill(cp, batch, global_offset, local_len, nullptr);
+  if (st != HS2_OK) return st;
+  cp.idx = idx;
+  cp.idx_stride = idx_stride;
+  cp.count = count;
+  cp.idx_out = idx_local;
+  cp.out_stride = idx_local_stride;
+  cp.count_out = count_local;
+  st = cuda_check(launch_cp_localize(cp, static_cast<cudaStream_t>(stream)), "selection localize");
   return st == HS2_OK ? ok() : st;
 }
 

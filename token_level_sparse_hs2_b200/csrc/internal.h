@@ -103,6 +103,8 @@ struct SparseParams {
   int32_t out_f32;
   uint32_t *status;
   int32_t idx_ready;        // idx / count were complete before the previous kernel started
+  int32_t allow_empty;      // count 0 is valid (a context shard holding none of the selection)
+  float *lse_out;           // [B*n_q, H] log-sum-exp of the attended scores, or null
 };
 
 // Cache append of n_q new rows per sequence (the last n_q rows of each sequence).
@@ -187,6 +189,37 @@ struct MergeParams {
   int32_t out_f32;
   float *lse;               // [groups, H] or null
 };
+
+// Context-parallel decode (a sequence's cache split by token range over ranks).
+constexpr int kCpMaxKeys = 16384;   // parts x topk composites merged in shared memory
+struct LseMergeParams {
+  int32_t n_parts, n_heads;
+  int64_t rows;
+  const float *part_o;      // [n_parts, rows, H, 128]
+  const float *part_lse;    // [n_parts, rows, H]
+  void *out;                // [rows, H, 128]
+  int32_t out_f32;
+  float *lse;               // [rows, H] or null
+};
+struct CpParams {
+  int32_t batch, n_parts, topk, window;
+  int64_t offset[HS2_MAX_BATCH];   // global position of the shard's first row, per sequence
+  int32_t local_len[HS2_MAX_BATCH];
+  int32_t global_len[HS2_MAX_BATCH];
+  const float *scores;
+  int64_t score_stride;
+  const int32_t *idx;       // [B, idx_stride]
+  int32_t idx_stride;
+  const int32_t *count;
+  uint64_t *keys;           // pack: [B, topk]; select: [n_parts, B, topk] (const)
+  int32_t *idx_out;         // select: [B, out_stride] global; localize: [B, out_stride] local
+  int32_t out_stride;
+  int32_t *count_out;
+};
+cudaError_t launch_lse_merge(const LseMergeParams &p, cudaStream_t s);
+cudaError_t launch_cp_pack(const CpParams &p, cudaStream_t s);
+cudaError_t launch_cp_select(const CpParams &p, cudaStream_t s);
+cudaError_t launch_cp_localize(const CpParams &p, cudaStream_t s);
 
 struct TensorMaps {
   CUtensorMap k, v;
