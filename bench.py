@@ -276,6 +276,61 @@ def bench_kv_bridge(hs2, dev, hbm, tf_burst, tokens=32768, d_model=4096, iters=1
             "note": "hidden states (%.0f MB) exceed L2; no flush" % (tokens * d_model * 2 / 1e6)}
 
 
+def bench_cp_shard(hs2, w, d, dev, world=8, iters=10):
+    """Context-parallel decode of this one-sequence workload over `world` ranks: the kernels of
+    one rank's block step (the last shard, which holds the window), timed on this GPU with the
+    all-gathers replaced by a local copy (only one GPU here: the NCCL exchanges are not timed)."""
+    from token_level_sparse_hs2_b200 import cp
+    T, H, L = int(w.kv_len[0]), w.n_heads, w.n_sparse
+    bounds = [T * k // world for k in range(world + 1)]
+    off, tl = bounds[-2], bounds[-1] - bounds[-2]
+    cache = hs2.KvCache(d["k"], d["v"], [int(w.kv_start[0]) + off], [tl], 1, H, d["k_scale"],
+                        d["v_scale"])
+    ws = torch.empty(hs2.workspace_size(cache, w.topk, min(w.window, tl)), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((1, 1, H, 128), dtype=torch.float32, device=dev)
+    outs = [torch.empty_like(out) for _ in range(L)]
+    sizes = []
+
+    def gather(x):
+        sizes.append(x.numel() * x.element_size())
+        return x.unsqueeze(0).expand((world,) + tuple(x.shape)).contiguous()
+
+    def step():
+        cp.cp_block_decode(cache, off, T, d["q_full"], d["q_sparse"], out, outs, ws, gather,
+                           topk=w.topk, window=w.window)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    # one step captured in a CUDA graph and replayed, so that the host's per-call cost (Python,
+    # argument checks) does not show in the device time
+    n0 = hs2.launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    launches = hs2.launch_count() - n0
+    graph.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(iters):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del graph
+    return {"world": world, "shard_tokens": tl, "us_per_rank_step": e0.elapsed_time(e1) / iters * 1e3,
+            "timing": "CUDA graph of one step, replayed %d times" % iters,
+            "library_launches_per_step": launches,
+            "allgathers_per_step": 2 + L, "bytes_per_rank_per_allgather": sizes[:2 + L],
+            "note": "one rank's kernels; the all-gathers (NCCL over NVLink) are replaced by a "
+                    "local copy on this one-GPU run and not timed"}
+
+
 def bench_block_select(hs2, cache, scores, w, dev, token_ms, block_size=64, iters=20):
     """Block-level selection (HySparse's granularity at the same budget) on the step's own
     scores, beside the token-level selection's traced time: pooling + per-row select."""
@@ -497,6 +552,8 @@ def main():
         line["e2e"] = e2e
     line["kv_append"] = bench_kv_append(hs2, dev, hbm)
     line["kv_bridge"] = bench_kv_bridge(hs2, dev, hbm, tf_burst)
+    if w.batch == 1 and w.n_q == 1 and int(w.kv_len[0]) >= 65536:
+        line["cp_decode"] = bench_cp_shard(hs2, w, d, dev)
     line["block_select"] = bench_block_select(hs2, cache, scores, w, dev, per["topk"])
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)

@@ -286,7 +286,8 @@ hs2_status hs2_cp_pack_candidates(const hs2_kv_view *kv, const int64_t *global_o
                                   uint64_t *keys, void *stream);
 
 /* The global selection from every shard's keys (device u64 [n_parts, batch, topk], n_parts x topk
- * <= 16384): with p = global_len[b] - 1 and nc = max(0, p - window + 1), all of [0, p] if
+ * <= 16384, part j being the shard that holds the j-th range of positions, each part's keys in
+ * position order as hs2_cp_pack_candidates writes them): with p = global_len[b] - 1 and nc = max(0, p - window + 1), all of [0, p] if
  * nc <= topk, else the topk largest keys' positions ascending, then [nc, p] -- what
  * hs2_topk_select gives on the whole context's scores. idx: device int32 [batch, idx_stride]
  * (global positions), count: device int32 [batch]. global_len: HOST [batch]. */

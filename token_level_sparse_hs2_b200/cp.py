@@ -13,6 +13,8 @@ lies in the union of the shards' own top-k. The kernels are the library's (see h
 
 Shapes: one sequence (batch 1), one decode query (n_q 1). Rank r holds global positions
 [offset, offset + T_local) as a KvCache of T_local rows; T_global is the whole context.
+The shards follow the ranks' order: rank r's positions all precede rank r + 1's (the merged
+selection is laid out shard by shard, so rank order is position order).
 """
 from __future__ import annotations
 

@@ -8,9 +8,11 @@
 //    (lse_merge_kernel), for the full layer and for every sparse layer;
 //  * the score of a position needs only the global lse, so after the first merge every rank
 //    scores its own positions; the top-k of the whole context is contained in the union of the
-//    shards' own top-k, so each rank packs its top-k (score, global position) pairs
-//    (cp_pack_kernel) and every rank merges all of them (cp_select_kernel) to the same global
-//    selection, ties to the lower position, window appended as on one GPU;
+//    shards' own top-k, so each rank packs its top-k (score, global position) pairs in position
+//    order (cp_pack_kernel) and every rank merges all of them (cp_select_kernel: a radix select
+//    of the exact topk-th largest, then the keys above it in list order, which is position
+//    order) to the same global selection, ties to the lower position, window appended as on
+//    one GPU;
 //  * each rank then attends to the selected positions it holds (cp_localize_kernel maps the
 //    ascending global selection to its contiguous local run).
 // "HySparse2: Hybrid Sparse Attention with Two-Level KV Sharing", bullet "Inference cost" (1M
@@ -54,38 +56,74 @@ __device__ __forceinline__ uint64_t cp_key(float score, int64_t g) {
   return ((uint64_t)__float_as_uint(score) << 32) | (uint64_t)(0xffffffffu - (uint32_t)g);
 }
 
-// One CTA per sequence: the shard's selected positions that are global candidates (position
-// below the global window) as packed keys, then empty slots up to topk.
-__global__ void __launch_bounds__(256) cp_pack_kernel(const __grid_constant__ CpParams P) {
+constexpr int kCpThreads = 512;
+constexpr int kCpWarps = kCpThreads / 32;
+
+// exclusive prefix sum over the CTA (kCpThreads threads) of one int per thread; *total = sum
+__device__ int cp_block_scan(int v, int *warp_sums, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = lane < kCpWarps ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < kCpWarps) warp_sums[lane] = s;
+  }
+  __syncthreads();
+  const int before = (warp ? warp_sums[warp - 1] : 0) + x - v;
+  *total = warp_sums[kCpWarps - 1];
+  __syncthreads();
+  return before;
+}
+
+// One CTA per sequence. The shard's selection idx is ascending and its global candidates
+// (positions below the global window) come first, so they are packed in position order into the
+// first slots; the remaining slots are empty (0).
+__global__ void __launch_bounds__(kCpThreads) cp_pack_kernel(const __grid_constant__ CpParams P) {
   __shared__ int n_s;
   griddep_launch_dependents();
   griddep_wait();
   const int b = blockIdx.x;
   const int64_t wstart = (int64_t)P.global_len[b] - P.window;   // first window position
-  const int cnt = min(__ldcg(P.count + b), P.idx_stride);
+  const int cnt = min(min(__ldcg(P.count + b), P.idx_stride), P.topk + P.window);
   const int32_t *idx = P.idx + (size_t)b * P.idx_stride;
   const float *s = P.scores + (size_t)b * P.score_stride;
   uint64_t *keys = P.keys + (size_t)b * P.topk;
   if (threadIdx.x == 0) n_s = 0;
   __syncthreads();
-  for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
+  int mine = 0;
+  for (int j = threadIdx.x; j < cnt; j += kCpThreads) {
     const int t = __ldcg(idx + j);
     const int64_t g = P.offset[b] + t;
-    if (t >= 0 && t < P.local_len[b] && g < wstart) {
-      const int slot = atomicAdd(&n_s, 1);
-      if (slot < P.topk) keys[slot] = cp_key(__ldcg(s + t), g);
+    if (t >= 0 && t < P.local_len[b] && g < wstart && j < P.topk) {
+      keys[j] = cp_key(__ldcg(s + t), g);
+      ++mine;
     }
   }
+  atomicAdd(&n_s, mine);
   __syncthreads();
-  for (int j = n_s + threadIdx.x; j < P.topk; j += blockDim.x) keys[j] = 0;
+  for (int j = n_s + threadIdx.x; j < P.topk; j += kCpThreads) keys[j] = 0;
 }
 
-constexpr int kCpThreads = 512;
-
-// One CTA per sequence: the topk largest of the n_parts x topk packed keys (bitonic sort in
-// shared memory), their positions in ascending order (a second bitonic sort), then the window.
+// One CTA per sequence: the exact topk-th largest key tau of the n_parts x topk keys by a radix
+// select on 8-bit digits from the top (stopping as soon as the bucket holds exactly the keys
+// still needed), then the keys >= tau kept in list order -- shard by shard, each shard's keys in
+// position order -- which is ascending position order; the window follows.
 __global__ void __launch_bounds__(kCpThreads) cp_select_kernel(const __grid_constant__ CpParams P) {
   extern __shared__ __align__(16) uint64_t cp_keys[];
+  __shared__ uint32_t hist[256];
+  __shared__ int warp_sums[kCpWarps];
+  __shared__ int bucket_s, above_s, inb_s;
   griddep_launch_dependents();
   griddep_wait();
   const int b = blockIdx.x;
@@ -98,94 +136,91 @@ __global__ void __launch_bounds__(kCpThreads) cp_select_kernel(const __grid_cons
     return;
   }
   const int n = P.n_parts * P.topk;
-  int np = 1;
-  while (np < n) np <<= 1;
-  for (int i = threadIdx.x; i < np; i += kCpThreads) {
-    uint64_t v = 0;
-    if (i < n) {
-      const int part = i / P.topk, j = i % P.topk;
-      v = __ldcg(P.keys + ((size_t)part * P.batch + b) * P.topk + j);
-    }
-    cp_keys[i] = v;
+  for (int i = threadIdx.x; i < n; i += kCpThreads) {
+    const int part = i / P.topk, j = i % P.topk;
+    cp_keys[i] = __ldcg(P.keys + ((size_t)part * P.batch + b) * P.topk + j);
   }
   __syncthreads();
-  for (int k = 2; k <= np; k <<= 1) {           // ascending bitonic sort
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < np; i += kCpThreads) {
-        const int x = i ^ j;
-        if (x > i) {
-          const uint64_t a = cp_keys[i], c = cp_keys[x];
-          if (((i & k) == 0) == (a > c)) {
-            cp_keys[i] = c;
-            cp_keys[x] = a;
+  uint64_t prefix = 0, mask = 0;
+  int need = P.topk;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    hist[threadIdx.x & 255] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kCpThreads) {
+      const uint64_t k = cp_keys[i];
+      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {   // bucket holding the need-th largest: one warp scans from the top
+      const int lane = threadIdx.x;
+      uint32_t c[8], sum = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        c[e] = hist[255 - (lane * 8 + e)];
+        sum += c[e];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t run = incl - sum;
+      if (run < (uint32_t)need && (uint32_t)need <= incl) {
+        for (int e = 0; e < 8; ++e) {
+          if (run + c[e] >= (uint32_t)need) {
+            bucket_s = 255 - (lane * 8 + e);
+            above_s = (int)run;
+            inb_s = (int)c[e];
+            break;
           }
+          run += c[e];
         }
       }
-      __syncthreads();
     }
+    __syncthreads();
+    need -= above_s;
+    prefix |= (uint64_t)bucket_s << shift;
+    mask |= (uint64_t)0xff << shift;
+    const bool whole = inb_s == need;   // every key of the bucket is kept
+    __syncthreads();
+    if (whole) break;
   }
-  // the topk largest are the last topk; their positions, padded to a power of two, sorted
-  int kp = 1;
-  while (kp < P.topk) kp <<= 1;
-  uint32_t *pos = reinterpret_cast<uint32_t *>(cp_keys);   // reuses the front of the buffer
-  uint32_t sel[HS2_MAX_TOPK / kCpThreads];
-  int ns = 0;
-  for (int i = threadIdx.x; i < kp; i += kCpThreads, ++ns)
-    sel[ns] = (i < P.topk) ? 0xffffffffu - (uint32_t)cp_keys[np - 1 - i] : 0xffffffffu;
-  __syncthreads();
-  ns = 0;
-  for (int i = threadIdx.x; i < kp; i += kCpThreads, ++ns) pos[i] = sel[ns];
-  __syncthreads();
-  for (int k = 2; k <= kp; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < kp; i += kCpThreads) {
-        const int x = i ^ j;
-        if (x > i) {
-          const uint32_t a = pos[i], c = pos[x];
-          if (((i & k) == 0) == (a > c)) {
-            pos[i] = c;
-            pos[x] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
+  // keys with (key & mask) >= prefix are the topk largest; keep them in list order
+  int run = 0;
+  for (int i0 = 0; i0 < n; i0 += kCpThreads) {
+    const int i = i0 + threadIdx.x;
+    const bool take = i < n && (cp_keys[i] & mask) >= prefix;
+    int tot;
+    const int pos = cp_block_scan(take ? 1 : 0, warp_sums, &tot);
+    if (take && run + pos < P.topk) out[run + pos] = (int32_t)(0xffffffffu - (uint32_t)cp_keys[i]);
+    run += tot;
   }
-  for (int i = threadIdx.x; i < P.topk; i += kCpThreads) out[i] = (int32_t)pos[i];
   for (int64_t t = nc + threadIdx.x; t <= p; t += kCpThreads) out[P.topk + (t - nc)] = (int32_t)t;
   if (threadIdx.x == 0) P.count_out[b] = (int32_t)(P.topk + (p - nc + 1));
 }
 
 // One CTA per sequence: the ascending global selection's positions inside this shard form one
-// contiguous run; it is copied out shifted to local positions (possibly empty).
-__global__ void __launch_bounds__(256) cp_localize_kernel(const __grid_constant__ CpParams P) {
-  __shared__ int lo_s, hi_s;
+// contiguous run [lo, lo + n); it is copied out shifted to local positions (possibly empty).
+__global__ void __launch_bounds__(kCpThreads) cp_localize_kernel(const __grid_constant__ CpParams P) {
+  __shared__ int warp_sums[kCpWarps];
   griddep_launch_dependents();
   griddep_wait();
   const int b = blockIdx.x;
   const int cnt = min(__ldcg(P.count + b), P.idx_stride);
   const int32_t *S = P.idx + (size_t)b * P.idx_stride;
   const int64_t g0 = P.offset[b], g1 = g0 + P.local_len[b];
-  if (threadIdx.x == 0) {
-    int lo = 0, hi = cnt;   // first entry >= g0
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (__ldcg(S + mid) < g0) lo = mid + 1;
-      else hi = mid;
-    }
-    int lo2 = lo, hi2 = cnt;   // first entry >= g1
-    while (lo2 < hi2) {
-      const int mid = (lo2 + hi2) >> 1;
-      if (__ldcg(S + mid) < g1) lo2 = mid + 1;
-      else hi2 = mid;
-    }
-    lo_s = lo;
-    hi_s = lo2;
+  int below = 0, inside = 0;
+  for (int j = threadIdx.x; j < cnt; j += kCpThreads) {
+    const int64_t g = __ldcg(S + j);
+    below += g < g0;
+    inside += g >= g0 && g < g1;
   }
-  __syncthreads();
-  const int lo = lo_s, n = hi_s - lo_s;
+  int lo, n;
+  cp_block_scan(below, warp_sums, &lo);
+  cp_block_scan(inside, warp_sums, &n);
   int32_t *out = P.idx_out + (size_t)b * P.out_stride;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) out[j] = (int32_t)(__ldcg(S + lo + j) - g0);
+  for (int j = threadIdx.x; j < n; j += kCpThreads) out[j] = (int32_t)(__ldcg(S + lo + j) - g0);
   if (threadIdx.x == 0) P.count_out[b] = n;
 }
 
@@ -199,7 +234,7 @@ cudaError_t launch_lse_merge(const LseMergeParams &p, cudaStream_t s) {
 }
 
 cudaError_t launch_cp_pack(const CpParams &p, cudaStream_t s) {
-  cudaError_t e = launch_pdl(cp_pack_kernel, p.batch, 256, 0, s, p);
+  cudaError_t e = launch_pdl(cp_pack_kernel, p.batch, kCpThreads, 0, s, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -214,7 +249,7 @@ cudaError_t launch_cp_select(const CpParams &p, cudaStream_t s) {
 }
 
 cudaError_t launch_cp_localize(const CpParams &p, cudaStream_t s) {
-  cudaError_t e = launch_pdl(cp_localize_kernel, p.batch, 256, 0, s, p);
+  cudaError_t e = launch_pdl(cp_localize_kernel, p.batch, kCpThreads, 0, s, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
