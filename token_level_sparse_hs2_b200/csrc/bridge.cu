@@ -7,15 +7,16 @@
 // projections, K_j = Proj_j^K(H_i^self), V_j = Proj_j^V(H_i^self) (here: linear maps, no bias).
 //
 // One dense GEMM [M, d] x [d, 256] -> [M, 256] (K and V side by side) on the fifth-generation
-// tensor cores, persistent over 128-row tiles:
-//   warp 5      TMA producer: a 128 x 64 tile of the hidden states and the 256 x 64 tile of
-//               the weights per k-block, kBrStages stages of 48 KB;
-//   warp 4      MMA issuer (one thread, M = 128, N = 256, K = 16 per instruction) and TMEM
-//               owner: two accumulators of 256 columns, so the epilogue of one tile overlaps
-//               the products of the next;
-//   warps 0..3  epilogue: warp w reads TMEM lanes 32 w .. + 31 (one output row per thread),
-//               rounds K and V to bf16 and writes the cache row of that token: bf16 as is, or
-//               e4m3 codes plus the row's scale (the same quantiser as the cache append).
+// tensor cores, persistent over units of two 128-row tiles that share each weight tile (the
+// weights are re-read from L2 for every unit and k-block, so sharing them cuts the bytes per
+// product by a third):
+//   warp 5      TMA producer: two 128 x 64 tiles of the hidden states and the 256 x 64 tile of
+//               the weights per k-block, kBrStages stages of 64 KB;
+//   warp 4      MMA issuer (one thread, M = 128, N = 256, K = 16 per instruction, one
+//               accumulator of 256 TMEM columns per tile of the unit) and TMEM owner;
+//   warps 0..3  epilogue: warp w reads TMEM lanes 32 w .. + 31 (one output row per thread and
+//               tile), rounds K and V to bf16 and writes the cache row of that token: bf16 as
+//               is, or e4m3 codes plus the row's scale (the same quantiser as the cache append).
 #include "common.cuh"
 #include "internal.h"
 #include "quant.cuh"
@@ -26,13 +27,14 @@ namespace hs2 {
 namespace {
 
 constexpr int kBrM = 128, kBrN = 256, kBrK = 64;
-constexpr int kBrStages = 4;
+constexpr int kBrPair = 2;                            // 128-row tiles per unit, sharing the weights
+constexpr int kBrStages = 3;
 constexpr int kBrABytes = kBrM * 128;                 // [128 rows][64 bf16], 128-byte swizzle
 constexpr int kBrBBytes = kBrN * 128;                 // [256 rows][64 bf16]
-constexpr int kBrStageBytes = kBrABytes + kBrBBytes;
+constexpr int kBrStageBytes = kBrPair * kBrABytes + kBrBBytes;
 constexpr int kBrWarpMma = 4, kBrWarpTma = 5;
 constexpr int kBrThreads = 6 * 32;
-constexpr uint32_t kBrCols = 2 * kBrN;
+constexpr uint32_t kBrCols = kBrPair * kBrN;          // one accumulator per tile of the unit
 
 struct BrSmem {
   uint8_t *stages;
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   BrSmem sm(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = (P.m + kBrM - 1) / kBrM;
+  const int n_tiles = (P.m + kBrPair * kBrM - 1) / (kBrPair * kBrM);   // units of kBrPair tiles
   const int nk = P.d_model / kBrK;
 
   if (threadIdx.x == 0) {
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&sm.acc_full[a]), 1);
       mbar_init(smem_u32(&sm.acc_empty[a]), 4);
-    }
+    }   // index 0 used: the unit's accumulators fill all of TMEM
     mbar_init(smem_u32(&sm.done[0]), 1);
     *sm.abort_flag = 0;
     fence_barrier_init();
@@ -159,8 +161,9 @@ __global__ void __launch_bounds__(kBrThreads, 1)
             uint8_t *st = sm.stages + s * kBrStageBytes;
             const uint32_t bar = smem_u32(&sm.full[s]);
             mbar_arrive_expect_tx(bar, kBrStageBytes);
-            tma_load_2d(smem_u32(st), &tm.h, bar, kb * kBrK, tile * kBrM);
-            tma_load_2d(smem_u32(st + kBrABytes), &tm.w, bar, kb * kBrK, 0);
+            for (int h = 0; h < kBrPair; ++h)
+              tma_load_2d(smem_u32(st + h * kBrABytes), &tm.h, bar, kb * kBrK, (tile * kBrPair + h) * kBrM);
+            tma_load_2d(smem_u32(st + kBrPair * kBrABytes), &tm.w, bar, kb * kBrK, 0);
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -173,8 +176,8 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     int it = 0, tl = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tl) {
-      const int a = tl & 1;
-      if (lane == 0 && tl >= 2 && !mbar_wait(smem_u32(&sm.acc_empty[a]), ((tl >> 1) & 1) ^ 1)) {
+      const int a = 0;
+      if (lane == 0 && tl >= 1 && !mbar_wait(smem_u32(&sm.acc_empty[a]), (tl & 1) ^ 1)) {
         br_fail(P, sm.abort_flag);
         ok = false;
       }
@@ -197,8 +200,10 @@ __global__ void __launch_bounds__(kBrThreads, 1)
           const uint32_t st = smem_u32(sm.stages + s * kBrStageBytes);
 #pragma unroll
           for (int k = 0; k < kBrK / 16; ++k)
-            umma_bf16(tmem + a * kBrN, umma_desc_sw128(st + k * 32, 1024),
-                      umma_desc_sw128(st + kBrABytes + k * 32, 1024), idesc, (kb | k) != 0);
+#pragma unroll
+            for (int h = 0; h < kBrPair; ++h)
+              umma_bf16(tmem + h * kBrN, umma_desc_sw128(st + h * kBrABytes + k * 32, 1024),
+                        umma_desc_sw128(st + kBrPair * kBrABytes + k * 32, 1024), idesc, (kb | k) != 0);
           umma_commit(smem_u32(&sm.empty[s]));
           if (kb == nk - 1) umma_commit(smem_u32(&sm.acc_full[a]));
         }
@@ -216,27 +221,29 @@ __global__ void __launch_bounds__(kBrThreads, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     int tl = 0;
     for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++tl) {
-      const int a = tl & 1;
+      const int a = 0;
       bool ok = true;
-      if (lane == 0 && !mbar_wait(smem_u32(&sm.acc_full[a]), (tl >> 1) & 1)) {
+      if (lane == 0 && !mbar_wait(smem_u32(&sm.acc_full[a]), tl & 1)) {
         br_fail(P, sm.abort_flag);
         ok = false;
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok || *sm.abort_flag) break;
       tc_fence_after();
-      const int r = tile * kBrM + warp * 32 + lane;   // row of the hidden-state matrix
-      const bool valid = r < P.m;
-      int64_t row = 0;
-      if (valid) {
-        const int b = r / P.n_q, i = r % P.n_q;
-        row = P.seq.start[b] + (int64_t)P.seq.len[b] - P.n_q + i;
+      for (int h = 0; h < kBrPair; ++h) {
+        const int r = (tile * kBrPair + h) * kBrM + warp * 32 + lane;   // row of the hidden states
+        const bool valid = r < P.m;
+        int64_t row = 0;
+        if (valid) {
+          const int b = r / P.n_q, i = r % P.n_q;
+          row = P.seq.start[b] + (int64_t)P.seq.len[b] - P.n_q + i;
+        }
+        const size_t rb = P.fp8 ? kHeadDim : kHeadDim * 2;   // bytes per cache row
+        store_row(lane_addr + h * kBrN, P.fp8, valid, static_cast<uint8_t *>(P.k) + row * rb,
+                  P.k_scale + row);
+        store_row(lane_addr + h * kBrN + 128, P.fp8, valid, static_cast<uint8_t *>(P.v) + row * rb,
+                  P.v_scale + row);
       }
-      const size_t rb = P.fp8 ? kHeadDim : kHeadDim * 2;   // bytes per cache row
-      store_row(lane_addr + a * kBrN, P.fp8, valid, static_cast<uint8_t *>(P.k) + row * rb,
-                P.k_scale + row);
-      store_row(lane_addr + a * kBrN + 128, P.fp8, valid, static_cast<uint8_t *>(P.v) + row * rb,
-                P.v_scale + row);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.acc_empty[a]));

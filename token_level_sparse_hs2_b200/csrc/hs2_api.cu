@@ -1186,7 +1186,7 @@ hs2_status hs2_kv_bridge(const hs2_kv_view *kv, const void *hidden, int32_t d_mo
   if ((st = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) != HS2_OK) return st;
   if ((st = cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev),
                        "SM count")) != HS2_OK) return st;
-  const int n_tiles = (int)((m + 127) / 128);
+  const int n_tiles = (int)((m + 255) / 256);   // units of two 128-row tiles
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((st = cuda_check(cudaMemsetAsync(workspace, 0, 4, s), "status clear")) != HS2_OK) return st;
   st = cuda_check(launch_kv_bridge(tm, bp, std::min(n_tiles, sms), s), "KV bridging");
