@@ -300,7 +300,10 @@ __global__ void __launch_bounds__(kThreadsTk) topk_hist_kernel(const __grid_cons
     if (hist[t]) atomicAdd(&gh[t], hist[t]);
 }
 
-__global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_constant__ TopkParams P) {
+// kRegs: a segment of a split row is held in registers (decode rows, a few long rows); the
+// variant without it (one CTA per row, many rows) keeps two CTAs resident per SM.
+template <bool kRegs>
+__global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(const __grid_constant__ TopkParams P) {
   extern __shared__ __align__(16) uint8_t tk_raw[];
   TkSmem &sm = *reinterpret_cast<TkSmem *>(tk_raw);
   griddep_launch_dependents();
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
   const int64_t s0 = (int64_t)sg * P.seg_len, s1 = min(nc, s0 + P.seg_len);
   // a short segment (the usual split case) is read into registers together with the histogram
   constexpr int kRegKeys = 32;
-  const bool in_regs = gh && P.seg_len <= kRegKeys * kThreadsTk;
+  const bool in_regs = kRegs && gh && P.seg_len <= kRegKeys * kThreadsTk;
   uint32_t rk[kRegKeys];
   if (in_regs) {
 #pragma unroll
@@ -375,21 +378,76 @@ __global__ void __launch_bounds__(kThreadsTk) topk_select_kernel(const __grid_co
       }
     });
   }
-  for (int64_t base = in_regs ? s1 : s0; base < s1; base += kThreadsTk * kUnroll) {
-    uint32_t k[kUnroll];
-    uint32_t take = 0;
+  if (!in_regs) {
+    // Each warp walks its own contiguous range of the segment 32 positions at a time and
+    // appends its candidates in order to its own share of the buffer (no CTA-wide barrier per
+    // step); the shares are then closed up in warp order, which is position order.
+    constexpr int kWarpCap = kCandCap / kWarpsTk;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t span = ((s1 - s0 + kWarpsTk * 32 - 1) / (kWarpsTk * 32)) * 32;
+    const int64_t w0 = s0 + warp * span, w1 = min(s1, w0 + span);
+    uint32_t *wkey = sm.key + warp * kWarpCap;
+    int32_t *widx = sm.idx + warp * kWarpCap;
+    int wcount = 0;
+    const unsigned below = (1u << lane) - 1u;
+    for (int64_t base = w0; base < w1; base += 32 * kUnroll) {
+      uint32_t k[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t t = base + u * kThreadsTk + threadIdx.x;
-      k[u] = t < s1 ? load_key(s, t) : 0u;
-      if (t < s1 && (int)(k[u] >> 21) >= B1) take |= 1u << u;
-    }
-    ordered_append<kUnroll>(take, sm, n_local, [&](int slot, int u) {
-      if (slot < kCandCap) {
-        sm.key[slot] = k[u];
-        sm.idx[slot] = (int32_t)(base + u * kThreadsTk + threadIdx.x);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t t = base + u * 32 + lane;
+        k[u] = t < w1 ? load_key(s, t) : 0u;
       }
-    });
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t t = base + u * 32 + lane;
+        const bool take = t < w1 && (int)(k[u] >> 21) >= B1;
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        if (take) {
+          const int slot = wcount + __popc(m & below);
+          if (slot < kWarpCap) {
+            wkey[slot] = k[u];
+            widx[slot] = (int32_t)t;
+          }
+        }
+        wcount += __popc(m);
+      }
+    }
+    if (lane == 0) sm.scan[warp] = wcount;
+    __syncthreads();
+    int pre = 0, tot = 0, over = 0;
+    for (int w = 0; w < kWarpsTk; ++w) {
+      const int c = sm.scan[w];
+      if (w < warp) pre += c;
+      tot += c;
+      over |= c > kWarpCap;
+    }
+    __syncthreads();
+    if (over) {
+      n_local = kCandCap + 1;   // a share overflowed: the exact fallback reads the row again
+    } else {
+      // close up the shares in warp order: every share is read into registers before any is
+      // written at its place
+      constexpr int kPerLane = kWarpCap / 32;
+      uint32_t kk[kPerLane];
+      int32_t ii[kPerLane];
+#pragma unroll
+      for (int q = 0; q < kPerLane; ++q) {
+        const int j = q * 32 + lane;
+        kk[q] = j < wcount ? wkey[j] : 0u;
+        ii[q] = j < wcount ? widx[j] : 0;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int q = 0; q < kPerLane; ++q) {
+        const int j = q * 32 + lane;
+        if (j < wcount) {
+          sm.key[pre + j] = kk[q];
+          sm.idx[pre + j] = ii[q];
+        }
+      }
+      n_local += tot;
+    }
+    __syncthreads();
   }
   int n;
   if (P.n_seg == 1) {
@@ -460,15 +518,19 @@ size_t topk_smem_bytes() { return sizeof(TkSmem); }
 
 cudaError_t launch_topk(const TopkParams &p, int n_rows, cudaStream_t s) {
   const size_t smem = sizeof(TkSmem);
-  cudaError_t e = cudaFuncSetAttribute(topk_select_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool regs = p.n_seg > 1;
+  cudaError_t e = regs ? cudaFuncSetAttribute(topk_select_kernel<true>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                       : cudaFuncSetAttribute(topk_select_kernel<false>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int grid = n_rows * p.n_seg;
   if (!p.hist && p.n_seg > 1) {
     e = launch_pdl(topk_hist_kernel, grid, kThreadsTk, 0, s, p);
     if (e != cudaSuccess) return e;
   }
-  e = launch_pdl(topk_select_kernel, grid, kThreadsTk, smem, s, p);
+  e = regs ? launch_pdl(topk_select_kernel<true>, grid, kThreadsTk, smem, s, p)
+           : launch_pdl(topk_select_kernel<false>, grid, kThreadsTk, smem, s, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
