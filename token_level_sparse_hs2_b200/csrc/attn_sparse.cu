@@ -10,8 +10,8 @@
 // 64-row tile (16-byte cp.async into the swizzled tile layout, two stages) and runs the
 // tensor-core online softmax on 16 heads x 16 rows of it. The token groups of a CTA merge in
 // shared memory; the splits of a row form one thread-block cluster and merge through
-// distributed shared memory, each CTA finishing a subset of the heads, so no partial result
-// goes through HBM.
+// distributed shared memory: each CTA pushes its partial of head h into the CTA that finishes
+// head h (one cluster barrier, then local reads), so no partial result goes through HBM.
 // merge_partials_kernel (one CTA per output group and head) serves the decode full layer.
 #include <cooperative_groups.h>
 
@@ -42,6 +42,10 @@ struct SpCfg {
   static constexpr size_t kRegion = ((size_t)kStages * kStageBytes > kMergeBytes)
                                         ? (size_t)kStages * kStageBytes : (kMergeBytes + 1023) / 1024 * 1024;
   static constexpr size_t kSmem = 1024 + kRegion + 2 * kStages * 8 + 16 + kPreTiles * kTile * 4;
+  // split rows (a thread-block cluster per row): every CTA of the cluster pushes its (M, L, O) of
+  // head h into the shared memory of CTA h % n_tsplit, at [h / n_tsplit][pusher][kPartRow]
+  static constexpr size_t kRecvBytes = (size_t)(16 * HG + 15) * kPartRow * 4;
+  static constexpr size_t kSmemSplit = kSmem + kRecvBytes;
 };
 
 // This warp's share of tile `it`: rows [w * RPW, (w+1) * RPW), cp.async into stage `st`, then
@@ -122,6 +126,9 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
     fence_barrier_init();
   }
   __syncthreads();
+  // split rows: announce this CTA to its cluster now; the matching wait comes just before the
+  // first push into another CTA's shared memory, long after every CTA has started
+  if (P.n_tsplit > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   // idx / count come from the selection kernel. When it ran two or more launches earlier
   // (idx_ready: sparse layers after the first), the index staging and the first gathers are
   // issued before the wait for the previous layer, overlapping its tail. Every layer lets the
@@ -266,6 +273,11 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
     }
   }
   __syncthreads();
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int ns = P.n_tsplit;
+  float *recv = reinterpret_cast<float *>(smem_raw + C::kSmem);
+  if (ns > 1) asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   for (int t = threadIdx.x; t < H * kHeadDim / 4; t += C::kThreads) {   // sum of the token groups
     const int h = t / (kHeadDim / 4), d4 = t % (kHeadDim / 4);
     const int hgh = h >> 4, rh = h & 15;
@@ -291,8 +303,8 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
         *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(P.out) + oi) =
             make_uint2(pack_bf16(O.x * inv, O.y * inv), pack_bf16(O.z * inv, O.w * inv));
       }
-    } else {
-      float *row = cpart + h * kPartRow;
+    } else {   // push into the owner of head h
+      float *row = cluster.map_shared_rank(recv, h % ns) + ((h / ns) * ns + ts) * kPartRow;
       reinterpret_cast<float4 *>(row + kPartO)[d4] = O;
       if (d4 == 0) {
         row[0] = hml[2 * h];
@@ -300,19 +312,17 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
       }
     }
   }
-  if (P.n_tsplit == 1) return;
-  // cluster merge: CTA `ts` of the row finishes heads ts, ts + n_tsplit, ... one warp per head,
-  // reading every CTA's (M, L, O) of that head from its shared memory
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
+  if (ns == 1) return;
+  // cluster merge: CTA `ts` of the row finishes heads ts, ts + n_tsplit, ..., one warp per head,
+  // from the (M, L, O) every CTA pushed into its shared memory. After this barrier no CTA touches
+  // another's shared memory, so each may leave when done.
   cluster.sync();
-  const int ns = P.n_tsplit;
   for (int h = ts + ns * warp; h < H; h += ns * C::kWarps) {
+    const float *part = recv + (h / ns) * ns * kPartRow;   // [pusher][kPartRow]
     float mj = -INFINITY, lj = 0.f;
     if (lane < ns) {
-      const float *rrow = cluster.map_shared_rank(cpart, lane) + h * kPartRow;
-      mj = rrow[0];
-      lj = rrow[1];
+      mj = part[lane * kPartRow];
+      lj = part[lane * kPartRow + 1];
     }
     float M = mj;
 #pragma unroll
@@ -322,23 +332,13 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < ns; j0 += 4) {   // four remote loads in flight at a time
-      float4 o[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        o[u] = (j0 + u < ns)
-                   ? reinterpret_cast<const float4 *>(cluster.map_shared_rank(cpart, j0 + u) + h * kPartRow + kPartO)[lane]
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float f = __shfl_sync(0xffffffffu, fj, (j0 + u) & 31);
-        if (j0 + u < ns) {
-          O.x += f * o[u].x;
-          O.y += f * o[u].y;
-          O.z += f * o[u].z;
-          O.w += f * o[u].w;
-        }
-      }
+    for (int j = 0; j < ns; ++j) {
+      const float f = __shfl_sync(0xffffffffu, fj, j);
+      const float4 o = reinterpret_cast<const float4 *>(part + j * kPartRow + kPartO)[lane];
+      O.x += f * o.x;
+      O.y += f * o.y;
+      O.z += f * o.z;
+      O.w += f * o.w;
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     if (P.lse_out && lane == 0)
@@ -352,7 +352,6 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
           make_uint2(pack_bf16(O.x * inv, O.y * inv), pack_bf16(O.z * inv, O.w * inv));
     }
   }
-  cluster.sync();   // no CTA leaves while another may still read its shared memory
 }
 
 // One CTA per (group, head, quarter of head_dim): 32 slot lanes x 8 lanes of 4 output dims,
@@ -434,9 +433,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __g
 template <int KV, int HG>
 cudaError_t launch_sparse_t(const SparseParams &p, cudaStream_t s) {
   using C = SpCfg<KV, HG>;
-  static_assert(C::kSmem <= 227 * 1024, "sparse shared memory");
+  static_assert(C::kSmemSplit <= 227 * 1024, "sparse shared memory");
   auto kern = sparse_gather_kernel<KV, HG>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemSplit);
   if (e != cudaSuccess) return e;
   const int grid = p.batch * p.n_q * p.n_tsplit;
   if (p.n_tsplit == 1) {
@@ -446,7 +445,7 @@ cudaError_t launch_sparse_t(const SparseParams &p, cudaStream_t s) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e != cudaSuccess) return e;
     }
-    e = launch_pdl_cluster(kern, grid, C::kThreads, C::kSmem, p.n_tsplit, s, p);
+    e = launch_pdl_cluster(kern, grid, C::kThreads, C::kSmemSplit, p.n_tsplit, s, p);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -457,7 +456,7 @@ template <int KV, int HG>
 int max_cluster_t() {
   using C = SpCfg<KV, HG>;
   auto kern = sparse_gather_kernel<KV, HG>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem) != cudaSuccess ||
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemSplit) != cudaSuccess ||
       cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
     return 1;
@@ -466,7 +465,7 @@ int max_cluster_t() {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cs);
     cfg.blockDim = dim3(C::kThreads);
-    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.dynamicSmemBytes = C::kSmemSplit;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cs;
