@@ -34,7 +34,7 @@ struct StreamCfg {
   // tile rows per pass-1 warp and pass-1 consumer warps: bf16 64 rows x 6 warps (registers
   // for a whole tile's scores); e4m3 32 rows x 8 warps (the widening wants more warps)
   static constexpr int kPass1Rows = (KV == kKvBf16) ? 64 : 32;
-  static constexpr int kPass1Warps = (KV == kKvBf16) ? 6 : 8;
+  static constexpr int kPass1Warps = (KV == kKvBf16) ? 6 : 4;
   static constexpr int kPass2Rows = 32;   // tile rows per pass-2 warp (all heads)
   static constexpr int kGroupWarps = (PASS == 0) ? (kTile / kPass1Rows) * HG : kTile / kPass2Rows;
   static constexpr int kGroups = (PASS == 0) ? kPass1Warps / kGroupWarps : 4 / kGroupWarps;
@@ -44,7 +44,7 @@ struct StreamCfg {
   static constexpr int kVBytes = (PASS == 0) ? kKBytes : 0;
   static constexpr int kScaleBytes = (KV == kKvFp8) ? (PASS == 0 ? 512 : 256) : 0;
   static constexpr int kStageBytes = (kKBytes + kVBytes + kScaleBytes + 1023) / 1024 * 1024;
-  static constexpr int kStages = (KV == kKvBf16) ? (PASS == 0 ? 5 : 4) : (PASS == 0 ? 8 : 6);
+  static constexpr int kStages = (KV == kKvBf16) ? (PASS == 0 ? 5 : 4) : (PASS == 0 ? 4 : 6);
   static constexpr uint32_t kTxBytes = kKBytes + kVBytes;
   static constexpr uint32_t kFullCount = (KV == kKvFp8) ? 33 : 1;
   // pass 1: the consumer warps' partials of a sequence merge in shared memory ([H][128] output
@@ -254,7 +254,7 @@ __device__ void flush_partial(const DecodeParams &P, int b, int hg, const WarpSo
 }
 
 template <int KV, int HG>
-__global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, 1)
+__global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, (KV == kKvBf16) ? 1 : 2)
     decode_pass1_kernel(const __grid_constant__ TensorMaps tm, const __grid_constant__ DecodeParams P) {
   using C = StreamCfg<KV, HG, 0>;
   constexpr int H = 16 * HG;

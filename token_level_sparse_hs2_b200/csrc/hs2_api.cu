@@ -434,7 +434,8 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   int sms = 0;
   hs2_status st = sm_count(&sms);
   if (st != HS2_OK) return st;
-  const int G = std::max(1, std::min({sms, P.total_tiles, kMaxStreamCtas}));
+  const int per_sm1 = P.kv_dtype == HS2_KV_BF16 ? 1 : 2;   // resident pass-1 CTAs per SM
+  const int G = std::max(1, std::min({per_sm1 * sms, P.total_tiles, kMaxStreamCtas}));
   // partial slots: 4 per (CTA, sequence) pair; CTA i owns tiles [i*T/G, (i+1)*T/G)
   const int T = P.total_tiles;
   auto cta_of = [&](int g) { return (int)(((int64_t)(g + 1) * G - 1) / T); };
