@@ -463,28 +463,31 @@ def main():
     # ---- end to end through the public API: host queries in, host results out, every step
     e2e = None
     if not a.no_e2e:
-        hq = d["q_full"].cpu().pin_memory()
-        hqs = [q.cpu().pin_memory() for q in d["q_sparse"]]
-        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        hos = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(L)]
-        hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-        hcnt = torch.empty(cnt.shape, dtype=cnt.dtype).pin_memory()
-        dq = torch.empty_like(d["q_full"])
-        dqs = [torch.empty_like(q) for q in d["q_sparse"]]
-        h2d = hq.numel() * 2 + sum(q.numel() * 2 for q in hqs)
-        d2h = ho.numel() * 2 * (1 + L) + hidx.numel() * 4 + hcnt.numel() * 4
+        # one pinned host buffer in and one out per step: the queries of every layer packed
+        # together, and the outputs, indices and counts written into one device buffer
+        qn = d["q_full"].numel()
+        hq_all = torch.cat([d["q_full"].reshape(-1)] + [q.reshape(-1) for q in d["q_sparse"]]) \
+            .cpu().pin_memory()
+        dq_all = torch.empty_like(hq_all, device=dev)
+        dq = dq_all[:qn].view(d["q_full"].shape)
+        dqs = [dq_all[(l + 1) * qn:(l + 2) * qn].view(d["q_sparse"][l].shape) for l in range(L)]
+        on = out.numel()
+        o_bytes, i_bytes, c_bytes = (1 + L) * on * 2, idx.numel() * 4, cnt.numel() * 4
+        dbuf = torch.empty(o_bytes + i_bytes + c_bytes, dtype=torch.uint8, device=dev)
+        o_all = dbuf[:o_bytes].view(torch.bfloat16)
+        eo = o_all[:on].view(out.shape)
+        eos = [o_all[(l + 1) * on:(l + 2) * on].view(out.shape) for l in range(L)]
+        eidx = dbuf[o_bytes:o_bytes + i_bytes].view(torch.int32).view(idx.shape)
+        ecnt = dbuf[o_bytes + i_bytes:].view(torch.int32).view(cnt.shape)
+        hbuf = torch.empty(dbuf.numel(), dtype=torch.uint8).pin_memory()
+        h2d = hq_all.numel() * 2
+        d2h = hbuf.numel()
 
         def e2e_step():
-            dq.copy_(hq, non_blocking=True)
-            for x, y in zip(dqs, hqs):
-                x.copy_(y, non_blocking=True)
-            hs2.block_decode(cache, dq, dqs, out, outs, lse, scores, idx, cnt, ws,
+            dq_all.copy_(hq_all, non_blocking=True)
+            hs2.block_decode(cache, dq, dqs, eo, eos, lse, scores, eidx, ecnt, ws,
                              topk=w.topk, window=w.window)
-            ho.copy_(out, non_blocking=True)
-            for x, y in zip(hos, outs):
-                x.copy_(y, non_blocking=True)
-            hidx.copy_(idx, non_blocking=True)
-            hcnt.copy_(cnt, non_blocking=True)
+            hbuf.copy_(dbuf, non_blocking=True)
 
         for _ in range(3):
             e2e_step()
