@@ -59,9 +59,22 @@ def test_short_contexts_keep_everything():
             assert np.array_equal(g["idx"][b, :T], np.arange(T))
 
 
-@pytest.mark.parametrize("topk,window", [(8, 4), (3, 1), (64, 0), (2048, 256)])
+@pytest.mark.parametrize("topk,window", [(8, 4), (3, 1), (64, 0), (2048, 256), (2048, 4096)])
 def test_budget_variants(topk, window):
-    w = decode(batch=2, lengths=(700, 3000), topk=topk, window=window, needles=2)
+    """Budgets up to the largest the C ABI accepts (topk 2,048, window 4,096)."""
+    lengths = (700, 3000) if window < 4096 else (7000, 9000)
+    w = decode(batch=2, lengths=lengths, topk=topk, window=window, needles=2)
+    g = H().run_block(w)
+    H().check_block(w, g)
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+def test_max_batch(kv_dtype):
+    """The largest batch the C ABI accepts (128 sequences), ragged lengths from shorter than the
+    budget (every position kept) to several thousand tokens."""
+    rng = np.random.default_rng(128)
+    lens = tuple(int(x) for x in rng.integers(60, 6000, size=128))
+    w = decode(batch=128, lengths=lens, n_heads=16, kv_dtype=kv_dtype, needles=1)
     g = H().run_block(w)
     H().check_block(w, g)
 

@@ -44,7 +44,11 @@ struct StreamCfg {
   static constexpr int kVBytes = (PASS == 0) ? kKBytes : 0;
   static constexpr int kScaleBytes = (KV == kKvFp8) ? (PASS == 0 ? 512 : 256) : 0;
   static constexpr int kStageBytes = (kKBytes + kVBytes + kScaleBytes + 1023) / 1024 * 1024;
-  static constexpr int kStages = (KV == kKvBf16) ? (PASS == 0 ? 5 : 4) : (PASS == 0 ? 4 : 6);
+  static constexpr int kStages = (KV == kKvBf16) ? (PASS == 0 ? 6 : 4) : (PASS == 0 ? 4 : 6);
+  // Stage s is refilled for steps s, s + kStages, ...; with kStages a multiple of kGroups all
+  // of those steps belong to one group, so a group never waits on a stage whose previous fill
+  // another group has not consumed yet (a parity wait cannot tell fill f from fill f + 2).
+  static_assert(kStages % kGroups == 0, "stages must be a multiple of the consumer groups");
   static constexpr uint32_t kTxBytes = kKBytes + kVBytes;
   static constexpr uint32_t kFullCount = (KV == kKvFp8) ? 33 : 1;
   // pass 1: the consumer warps' partials of a sequence merge in shared memory ([H][128] output
