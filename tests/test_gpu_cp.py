@@ -135,3 +135,12 @@ def test_cp_short_context_keeps_everything():
     res = run_cp(w, bounds, w.topk, w.window)
     assert int(res[0]["count"][0]) == 900
     check(w, bounds, res, w.topk, w.window)
+
+
+def test_cp_shards_starting_inside_tiles():
+    """Shard boundaries that are not multiples of the 64-row tile, including a one-token shard
+    and the window split over two shards."""
+    w = workload(10_000, H=32, needles=8)
+    bounds = [0, 37, 38, 5001, 9_930, 10_000]
+    res = run_cp(w, bounds, w.topk, w.window)
+    check(w, bounds, res, w.topk, w.window)

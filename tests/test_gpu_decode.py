@@ -175,3 +175,15 @@ def test_config2_full_size_fp8():
     H().check_block(w, g)
     sel = set(g["idx"][0, :g["count"][0]].tolist())
     assert set(w.needle_pos[0].tolist()) <= sel
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+def test_lengths_at_tile_and_budget_edges(kv_dtype):
+    """One-token and two-token contexts, lengths at the 64-row tile edges, and the budget edge
+    (1,151 keeps everything, 1,152 = budget, 1,153 selects)."""
+    lens = (1, 2, 63, 64, 65, 127, 128, 129, 1151, 1152, 1153, 4097)
+    w = decode(batch=len(lens), lengths=lens, n_heads=32, kv_dtype=kv_dtype, needles=0)
+    g = H().run_block(w)
+    H().check_block(w, g)
+    for b, T in enumerate(lens):
+        assert g["count"][b] == min(T, 1152)

@@ -83,3 +83,14 @@ def test_config4_prefill_full_size():
     for j, r in enumerate(rows):
         p = int(r)
         assert g["count"][j] == min(p + 1, 1152)
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+def test_many_chunked_sequences(kv_dtype):
+    """Twelve sequences of 37 queries each (the last blocks of every sequence partial), ragged
+    contexts from just above the query count to several thousand tokens."""
+    lens = (37, 40, 101, 700, 1300, 2600, 64, 65, 129, 4000, 1153, 900)
+    w = chunk(batch=len(lens), n_q=37, lengths=lens, kv_dtype=kv_dtype, n_heads=16,
+              topk=128, window=32, needles=1)
+    g = H().run_block(w)
+    H().check_block(w, g, topk=128, window=32)
