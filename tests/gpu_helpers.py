@@ -17,7 +17,7 @@ O_TOL = {"bf16": 1e-2, "fp8": 3e-2}
 
 
 def run_block(w, out_dtype=torch.float32, topk=None, window=None, ws_fill=None, n_sparse=None,
-              stream=None, rows=None):
+              stream=None, rows=None, scale=None):
     """Runs the block on the GPU. With `rows`, only those flat query rows are copied back and
     the returned arrays are indexed by position in `rows`."""
     topk = w.topk if topk is None else topk
@@ -41,7 +41,7 @@ def run_block(w, out_dtype=torch.float32, topk=None, window=None, ws_fill=None, 
     if ws_fill is not None:
         ws.fill_(ws_fill)
     hs2.block_decode(cache, d["q_full"], d["q_sparse"][:L], out_full, out_sp, lse, scores, idx,
-                     count, ws, topk=topk, window=window, stream=stream)
+                     count, ws, topk=topk, window=window, scale=scale, stream=stream)
     hs2.read_device_status(ws, stream)
     torch.cuda.synchronize()
     if rows is None:
@@ -67,7 +67,7 @@ def check_scores(w, rows, s_gpu, s_ref):
         assert not bad.any(), (r, int(np.argmax(bad)), g[bad][:4], ref[bad][:4])
 
 
-def check_block(w, gpu, rows=None, topk=None, window=None, check_sparse=True):
+def check_block(w, gpu, rows=None, topk=None, window=None, check_sparse=True, scale=None):
     """Full comparison of a GPU block run against the oracle on the listed rows."""
     topk = w.topk if topk is None else topk
     window = w.window if window is None else window
@@ -77,7 +77,7 @@ def check_block(w, gpu, rows=None, topk=None, window=None, check_sparse=True):
     else:
         rows = np.arange(w.n_rows) if rows is None else np.asarray(rows)
         pos = rows
-    o_ref, lse_ref, s_ref = oracle.full_attn(w, rows=rows)
+    o_ref, lse_ref, s_ref = oracle.full_attn(w, rows=rows, scale=scale)
     tol = O_TOL[w.kv_dtype]
     err = np.abs(gpu["o_full"][pos] - o_ref).max()
     assert err <= tol, f"O_full max-abs {err}"
@@ -110,7 +110,7 @@ def check_block(w, gpu, rows=None, topk=None, window=None, check_sparse=True):
     if check_sparse:
         cnt = gpu["count"][pos]
         for l in range(len(gpu["o_sparse"])):
-            ref = oracle.sparse_attn(w, w.q_sparse[l], rows, gpu["idx"][pos], cnt)
+            ref = oracle.sparse_attn(w, w.q_sparse[l], rows, gpu["idx"][pos], cnt, scale)
             err = np.abs(gpu["o_sparse"][l][pos] - ref).max()
             assert err <= tol, f"sparse layer {l} max-abs {err}"
     return dict(o_ref=o_ref, lse_ref=lse_ref, s_ref=s_ref)

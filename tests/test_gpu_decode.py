@@ -187,3 +187,51 @@ def test_lengths_at_tile_and_budget_edges(kv_dtype):
     H().check_block(w, g)
     for b, T in enumerate(lens):
         assert g["count"][b] == min(T, 1152)
+
+
+def scatter(w, seed):
+    """The same sequences at permuted cache positions with junk rows between and after them,
+    so that any read outside a sequence's own rows would change the result."""
+    import copy
+    from workloads import f32_to_bf16_bits
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(w.batch)
+    gaps = rng.integers(1, 300, size=w.batch)
+    rows = int(w.kv_len.astype(np.int64).sum() + gaps.sum() + 77)
+    if w.kv_dtype == "bf16":
+        junk = lambda: f32_to_bf16_bits((rng.standard_normal((rows, 128)) * 30).astype(np.float32))
+    else:
+        junk = lambda: rng.integers(0, 0x7e, size=(rows, 128)).astype(np.uint8)
+    k, v = junk(), junk()
+    ks = vs = None
+    if w.kv_dtype == "fp8":
+        ks = (rng.random(rows) * 10).astype(np.float32)
+        vs = (rng.random(rows) * 10).astype(np.float32)
+    start = np.zeros(w.batch, dtype=np.int64)
+    pos = 0
+    for b in order:
+        pos += int(gaps[b])
+        start[b] = pos
+        s0, n = int(w.kv_start[b]), int(w.kv_len[b])
+        k[pos:pos + n], v[pos:pos + n] = w.k[s0:s0 + n], w.v[s0:s0 + n]
+        if ks is not None:
+            ks[pos:pos + n], vs[pos:pos + n] = w.k_scale[s0:s0 + n], w.v_scale[s0:s0 + n]
+        pos += n
+    w2 = copy.copy(w)
+    w2.k, w2.v, w2.k_scale, w2.v_scale, w2.kv_start = k, v, ks, vs, start
+    return w2
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8"])
+def test_scattered_sequences_and_custom_scale(kv_dtype):
+    """Sequences at permuted, gapped cache positions surrounded by junk rows, and a softmax scale
+    other than 1/sqrt(128): decode rows and 9-query chunks."""
+    base = decode(batch=5, lengths=(3000, 700, 5000, 129, 2222), kv_dtype=kv_dtype, needles=2)
+    w = scatter(base, 5)
+    g = H().run_block(w, scale=0.05)
+    H().check_block(w, g, scale=0.05)
+    base = decode(batch=3, n_q=9, lengths=(900, 2100, 40), kv_dtype=kv_dtype, needles=1,
+                  topk=256, window=32)
+    w = scatter(base, 6)
+    g = H().run_block(w, scale=0.05)
+    H().check_block(w, g, scale=0.05)
