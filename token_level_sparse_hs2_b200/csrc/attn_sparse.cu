@@ -360,7 +360,7 @@ constexpr int kMergeThreads = 256;
 constexpr int kMergeChunks = 4;
 
 __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __grid_constant__ MergeParams P) {
-  __shared__ float red_m[32];
+  __shared__ float red_m[kMergeThreads / 32];
   __shared__ float red_l[32];
   __shared__ float4 red_o[32][8];
   const int ch = blockIdx.x % kMergeChunks;
@@ -377,49 +377,44 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __g
   griddep_wait();   // partials come from the previous kernel
   const int H = P.n_heads;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // one pass: slot lane sl folds slots sl, sl + 32, ... into a running (max, sum, output),
-  // rescaling when the max grows; the 32 slot lanes are then combined the same way
+  float m = -INFINITY;
+  for (int i = threadIdx.x; i < n; i += kMergeThreads)
+    m = fmaxf(m, __ldcg(P.part + ((size_t)(s0 + i) * H + h) * kPartRow));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) red_m[w] = m;
+  __syncthreads();
+  float M = red_m[0];
+#pragma unroll
+  for (int i = 1; i < kMergeThreads / 32; ++i) M = fmaxf(M, red_m[i]);
   const int sl = w * 4 + (lane >> 3), dq = lane & 7;   // slot lane 0..31, dim quad 0..7
-  float m = -INFINITY, L = 0.f;
+  float L = 0.f;
   float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 2
   for (int i = sl; i < n; i += 32) {
     const float *row = P.part + ((size_t)(s0 + i) * H + h) * kPartRow;
     const float mi = __ldcg(row);
-    const float li = __ldcg(row + 1);
+    const float f = (mi == -INFINITY) ? 0.f : fast_exp2(mi - M);
+    L += f * __ldcg(row + 1);
     const float4 o = __ldcg(reinterpret_cast<const float4 *>(row + kPartO) + ch * 8 + dq);
-    if (mi == -INFINITY) continue;
-    const float mn = fmaxf(m, mi);
-    const float a = (m == -INFINITY) ? 0.f : fast_exp2(m - mn), f = fast_exp2(mi - mn);
-    L = a * L + f * li;
-    O.x = a * O.x + f * o.x;
-    O.y = a * O.y + f * o.y;
-    O.z = a * O.z + f * o.z;
-    O.w = a * O.w + f * o.w;
-    m = mn;
+    O.x += f * o.x;
+    O.y += f * o.y;
+    O.z += f * o.z;
+    O.w += f * o.w;
   }
   red_o[sl][dq] = O;
-  if (dq == 0) {
-    red_m[sl] = m;
-    red_l[sl] = L;
-  }
+  if (dq == 0) red_l[sl] = L;
   __syncthreads();
   if (threadIdx.x < 8) {
-    float M = -INFINITY;
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) M = fmaxf(M, red_m[k]);
     float Lt = 0.f;
     float4 Ot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
     for (int k = 0; k < 32; ++k) {
-      const float mk = red_m[k];
-      if (mk == -INFINITY) continue;
-      const float f = fast_exp2(mk - M);
-      Lt += f * red_l[k];
-      Ot.x += f * red_o[k][threadIdx.x].x;
-      Ot.y += f * red_o[k][threadIdx.x].y;
-      Ot.z += f * red_o[k][threadIdx.x].z;
-      Ot.w += f * red_o[k][threadIdx.x].w;
+      Lt += red_l[k];
+      Ot.x += red_o[k][threadIdx.x].x;
+      Ot.y += red_o[k][threadIdx.x].y;
+      Ot.z += red_o[k][threadIdx.x].z;
+      Ot.w += red_o[k][threadIdx.x].w;
     }
     const float inv = 1.f / Lt;
     const size_t oi = ((size_t)grp * H + h) * kHeadDim + ch * 32 + 4 * threadIdx.x;
