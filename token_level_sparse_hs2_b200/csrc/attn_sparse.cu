@@ -13,6 +13,7 @@
 // distributed shared memory: each CTA pushes its partial of head h into the CTA that finishes
 // head h (one cluster barrier, then local reads), so no partial result goes through HBM.
 // merge_partials_kernel (one CTA per output group and head) serves the decode full layer.
+#include <algorithm>
 #include <cooperative_groups.h>
 
 #include "attn_pipeline.cuh"
@@ -354,15 +355,20 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
   }
 }
 
-// One CTA per (group, head, quarter of head_dim): 32 slot lanes x 8 lanes of 4 output dims,
-// float4 loads, so a group with many slots still spreads over 4 * heads CTAs.
+// CTAs per (group, head, part of head_dim): slot lanes x lanes of 4 output dims, float4 loads,
+// so a group with many slots still spreads over several CTAs per head.
 constexpr int kMergeThreads = 256;
-constexpr int kMergeChunks = 4;
 
+// CHUNKS CTAs per (group, head), each owning 128 / CHUNKS output dims: 4 for a few partials per
+// group (fewer CTAs), 8 for many (more slot lanes, shorter chains of loads per lane).
+template <int CHUNKS>
 __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __grid_constant__ MergeParams P) {
+  constexpr int kMergeChunks = CHUNKS;
+  constexpr int kMergeQuads = 128 / 4 / kMergeChunks;        // float4 columns per CTA
+  constexpr int kMergeLanes = kMergeThreads / kMergeQuads;   // slot lanes
   __shared__ float red_m[kMergeThreads / 32];
-  __shared__ float red_l[32];
-  __shared__ float4 red_o[32][8];
+  __shared__ float red_l[kMergeLanes];
+  __shared__ float4 red_o[kMergeLanes][kMergeQuads];
   const int ch = blockIdx.x % kMergeChunks;
   const int grp = blockIdx.x / kMergeChunks / P.n_heads, h = blockIdx.x / kMergeChunks % P.n_heads;
   int s0, n;
@@ -387,16 +393,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __g
   float M = red_m[0];
 #pragma unroll
   for (int i = 1; i < kMergeThreads / 32; ++i) M = fmaxf(M, red_m[i]);
-  const int sl = w * 4 + (lane >> 3), dq = lane & 7;   // slot lane 0..31, dim quad 0..7
+  const int sl = threadIdx.x / kMergeQuads, dq = threadIdx.x % kMergeQuads;   // slot lane, dim quad
   float L = 0.f;
   float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 2
-  for (int i = sl; i < n; i += 32) {
+  for (int i = sl; i < n; i += kMergeLanes) {
     const float *row = P.part + ((size_t)(s0 + i) * H + h) * kPartRow;
     const float mi = __ldcg(row);
     const float f = (mi == -INFINITY) ? 0.f : fast_exp2(mi - M);
     L += f * __ldcg(row + 1);
-    const float4 o = __ldcg(reinterpret_cast<const float4 *>(row + kPartO) + ch * 8 + dq);
+    const float4 o = __ldcg(reinterpret_cast<const float4 *>(row + kPartO) + ch * kMergeQuads + dq);
     O.x += f * o.x;
     O.y += f * o.y;
     O.z += f * o.z;
@@ -405,11 +411,11 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __g
   red_o[sl][dq] = O;
   if (dq == 0) red_l[sl] = L;
   __syncthreads();
-  if (threadIdx.x < 8) {
+  if (threadIdx.x < kMergeQuads) {
     float Lt = 0.f;
     float4 Ot = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
+    for (int k = 0; k < kMergeLanes; ++k) {
       Lt += red_l[k];
       Ot.x += red_o[k][threadIdx.x].x;
       Ot.y += red_o[k][threadIdx.x].y;
@@ -417,7 +423,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_partials_kernel(const __g
       Ot.w += red_o[k][threadIdx.x].w;
     }
     const float inv = 1.f / Lt;
-    const size_t oi = ((size_t)grp * H + h) * kHeadDim + ch * 32 + 4 * threadIdx.x;
+    const size_t oi = ((size_t)grp * H + h) * kHeadDim + ch * (4 * kMergeQuads) + 4 * threadIdx.x;
     if (P.out_f32) {
       *reinterpret_cast<float4 *>(reinterpret_cast<float *>(P.out) + oi) =
           make_float4(Ot.x * inv, Ot.y * inv, Ot.z * inv, Ot.w * inv);
@@ -484,7 +490,12 @@ int max_cluster_t() {
 
 
 cudaError_t launch_merge(const MergeParams &p, cudaStream_t s) {
-  cudaError_t e = launch_pdl(merge_partials_kernel, p.n_groups * p.n_heads * kMergeChunks, kMergeThreads, 0, s, p);
+  int most = p.n_fixed;   // partials of the largest group
+  if (p.by_seq)
+    for (int g = 0; g < p.n_groups; ++g) most = std::max(most, p.seq.item_begin[g + 1] - p.seq.item_begin[g]);
+  cudaError_t e = most > 64
+      ? launch_pdl(merge_partials_kernel<8>, p.n_groups * p.n_heads * 8, kMergeThreads, 0, s, p)
+      : launch_pdl(merge_partials_kernel<4>, p.n_groups * p.n_heads * 4, kMergeThreads, 0, s, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
