@@ -201,3 +201,22 @@ def test_block_selection_argument_checks(L):
                                   idx.data_ptr(), 1000, cnt.data_ptr(), ctypes.c_void_p(256),
                                   1 << 20, None)
     assert st == 1 and b"idx_stride" in L.hs2_last_error()
+
+
+def test_context_parallel_argument_checks(L):
+    c = cpu_cache(batch=1, lens=(5000,))
+    P = ctypes.c_void_p
+    ws = P(256)
+    # NULL outputs, a bad scale, a short score stride, bad merge shapes: refused before any launch
+    assert L.hs2_full_attn(c.ref(), P(256), ctypes.c_float(0.088), None, 1, P(256), ws,
+                           1 << 20, None) == 1
+    assert L.hs2_full_attn(c.ref(), P(256), ctypes.c_float(-1.0), P(256), 1, P(256), ws,
+                           1 << 20, None) == 1
+    assert L.hs2_score_pass(c.ref(), P(256), ctypes.c_float(0.088), P(256), P(256), 100, ws,
+                            1 << 20, None) == 1
+    assert b"score_stride" in L.hs2_last_error()
+    assert L.hs2_lse_merge(0, 1, 32, P(256), P(256), P(256), 1, None, None) == 1
+    assert L.hs2_cp_merge_select(32, 1, (ctypes.c_int32 * 1)(5000), P(256), 1024, 128, P(256),
+                                 1152, P(256), None) == 2          # 32 x 1024 keys: too many
+    assert L.hs2_cp_localize(1, (ctypes.c_int64 * 1)(4000), (ctypes.c_int32 * 1)(1000), P(256),
+                             1152, P(256), P(256), 100, P(256), None) == 1

@@ -978,9 +978,11 @@ hs2_status hs2_full_attn(const hs2_kv_view *kv, const void *q, float softmax_sca
   if (kv->n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "hs2_full_attn is for decode (n_q = 1)");
   Plan P;
   make_plan(kv, P);
-  float dummy_scores = 0.f;   // not written: the score pass does not run
-  if ((st = check_full_args(P, q, softmax_scale, out, out_dtype, lse, &dummy_scores, P.max_p + 1)) != HS2_OK)
-    return st;
+  if (!q || !out || !lse) return fail(HS2_ERR_INVALID_ARG, "q / out / lse is NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(HS2_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
+  if (!valid_scale(softmax_scale)) return fail(HS2_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (out_dtype != HS2_OUT_BF16 && out_dtype != HS2_OUT_F32)
+    return fail(HS2_ERR_INVALID_ARG, "out_dtype %d", out_dtype);
   if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
   TensorMaps tm;
   if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
@@ -998,10 +1000,12 @@ hs2_status hs2_score_pass(const hs2_kv_view *kv, const void *q, float softmax_sc
   if (kv->n_q != 1) return fail(HS2_ERR_UNSUPPORTED, "hs2_score_pass is for decode (n_q = 1)");
   Plan P;
   make_plan(kv, P);
-  int dummy_out = 0;
-  if ((st = check_full_args(P, q, softmax_scale, q, HS2_OUT_F32, lse, scores, score_stride)) != HS2_OK)
-    return st;
-  (void)dummy_out;
+  if (!q || !lse || !scores) return fail(HS2_ERR_INVALID_ARG, "q / lse / scores is NULL");
+  if (!aligned16(q)) return fail(HS2_ERR_INVALID_ARG, "q must be 16-byte aligned");
+  if (!valid_scale(softmax_scale)) return fail(HS2_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (score_stride < P.max_p + 1)
+    return fail(HS2_ERR_INVALID_ARG, "score_stride %lld < %lld", (long long)score_stride,
+                (long long)(P.max_p + 1));
   if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
   TensorMaps tm;
   if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
