@@ -345,3 +345,35 @@ def test_kv_bridge_selector_weights_copy_features(oracle_lib):
     hb = bf16_bits_to_f32(h).astype(np.float64)
     assert np.array_equal(k, hb[:, 0:256:2])
     assert np.array_equal(v, -hb[:, 1:129])
+
+
+# ------------------------------------------------------------------ context-parallel decomposition
+
+def test_attention_over_disjoint_shards_merges_to_the_whole(oracle_lib):
+    """The reading behind context-parallel decode, pinned in the oracle: softmax attention over a
+    union of disjoint position sets is the log-sum-exp merge of the parts (closed form:
+    lse = log sum_j e^{lse_j}, O = sum_j e^{lse_j - lse} O_j), and the whole context's scores
+    under the merged lse are each shard's scores under that lse."""
+    import copy
+    w = small(batch=1, lengths=(900,), needles=2, n_heads=4)
+    o_ref, lse_ref, s_ref = oracle_lib.full_attn(w)
+    parts = []
+    for a, b in ((0, 333), (333, 899), (899, 900)):
+        ws = copy.copy(w)
+        ws.kv_start = np.array([int(w.kv_start[0]) + a], dtype=np.int64)
+        ws.kv_len = np.array([b - a], dtype=np.int32)
+        o, lse, _ = oracle_lib.full_attn(ws)
+        parts.append((o, lse))
+    L = np.stack([p[1] for p in parts])                       # [3, 1, H]
+    M = L.max(axis=0)
+    wgt = np.exp(L - M)
+    lse = M + np.log(wgt.sum(axis=0))
+    O = sum(wgt[j][..., None] * parts[j][0] for j in range(3)) / wgt.sum(axis=0)[..., None]
+    assert np.allclose(lse, lse_ref, rtol=0, atol=1e-12)
+    assert np.allclose(O, o_ref, rtol=0, atol=1e-12)
+    # scores of a shard under the merged lse equal the whole context's scores there
+    kd = dense_f64(w, "k").numpy()
+    q = q_f64(w.q_full).reshape(w.n_heads, 128)
+    logits = (q @ kd[:900].T) / math.sqrt(128)
+    s = np.exp(logits - lse.reshape(-1, 1)).sum(axis=0)
+    assert np.allclose(s, s_ref[0, :900], rtol=1e-12, atol=0)
