@@ -529,6 +529,8 @@ hs2_status run_topk(const hs2_kv_view *kv, const Plan &P, const float *scores,
   tp.score_stride = score_stride;
   tp.n_seg = P.n_seg;
   tp.seg_len = P.seg_len;
+  // rows split over at most 8 segments whose keys fit in registers: one cluster per row
+  tp.cluster = (P.n_seg > 1 && P.n_seg <= 8 && P.seg_len <= 32 * 512) ? 1 : 0;
   if (P.n_seg > 1) {
     if (hist_ready) tp.hist = sc.hist;
     else tp.hist_ws = sc.hist;

@@ -144,6 +144,7 @@ struct TopkParams {
   const uint32_t *hist;     // [B*n_q, kHistBins] top-digit counts from the score pass, or null
   uint32_t *hist_ws;        // [B*n_q, kHistBins] built here when hist is null and n_seg > 1
   int32_t n_seg, seg_len;
+  int32_t cluster;          // 1: the n_seg (<= 8) segments of a row are one thread-block cluster
   uint32_t *cand_key;       // [B*n_q, cand_cap] (n_seg > 1)
   int32_t *cand_idx;
   int32_t cand_cap;

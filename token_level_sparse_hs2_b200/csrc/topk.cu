@@ -16,10 +16,12 @@
 //  3. in shared memory: the exact threshold key tau (digits 20..10, 9..0), how many keys equal
 //     to tau are taken (the lowest indices: a radix select on the index); one more ordered
 //     compaction keeps the selected candidates in ascending order, and the window is appended.
-// Long rows are split over several CTAs (segments) that compact into a global buffer and record
-// where their run starts; the last segment to arrive lays the runs out in segment order and
-// finishes the row. If the compacted set does not fit (many equal scores),
+// Long rows are split over several CTAs (segments). Up to 8 segments form a thread-block
+// cluster and segment 0 gathers the runs from the others' shared memory; more segments compact
+// into a global buffer and record where their run starts, and the last segment to arrive lays
+// the runs out in segment order. Either way one CTA finishes the row. If the compacted set does not fit (many equal scores),
 // the finishing CTA falls back to exact digit passes and an ordered scan over the whole row.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -452,6 +454,39 @@ __global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(
   int n;
   if (P.n_seg == 1) {
     n = n_local;
+  } else if (P.cluster) {
+    // the row's segments form one thread-block cluster: segment 0 gathers the others' runs from
+    // their shared memory in segment order (its own run is already in place) and finishes
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    if (threadIdx.x == 0) sm.last = n_local;          // this segment's count, for rank 0
+    cluster.sync();
+    n = 0;
+    if (sg == 0) {
+      const int ns = P.n_seg;
+      const int cnt = threadIdx.x < ns ? *cluster.map_shared_rank(&sm.last, (int)threadIdx.x) : 0;
+      int tot;
+      const int pre = block_excl_scan(cnt, sm.warp_sums, &tot);
+      if (threadIdx.x < ns) sm.seg_pre[threadIdx.x] = pre;
+      __syncthreads();
+      n = tot;
+      if (n <= kCandCap) {
+        for (int j = sm.seg_pre[1 < ns ? 1 : 0] + threadIdx.x; j < n; j += kThreadsTk) {
+          int lo = 1, hi = ns - 1;   // the last segment starting at or before j
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sm.seg_pre[mid] <= j) lo = mid;
+            else hi = mid - 1;
+          }
+          const int off = j - sm.seg_pre[lo];
+          sm.key[j] = cluster.map_shared_rank(sm.key, lo)[off];
+          sm.idx[j] = cluster.map_shared_rank(sm.idx, lo)[off];
+        }
+      }
+      __syncthreads();
+    }
+    cluster.sync();   // no segment leaves while rank 0 may still read its shared memory
+    if (sg != 0) return;
   } else {
     // publish this segment's candidates with one global reservation and record where they
     // went, so that the finishing CTA can lay the segments out in position order
@@ -506,7 +541,7 @@ __global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(
     }
   }
   // 4. finish
-  const bool fits = (P.n_seg == 1) ? (n <= kCandCap) : (n <= kCandCap && n <= P.cand_cap);
+  const bool fits = (P.n_seg == 1 || P.cluster) ? (n <= kCandCap) : (n <= kCandCap && n <= P.cand_cap);
   if (fits) finish_from_smem(sm, n, B1, above, P.topk, out);
   else finish_from_global(sm, s, nc, B1, above, P.topk, out);
   // 5. the forced window
@@ -529,8 +564,11 @@ cudaError_t launch_topk(const TopkParams &p, int n_rows, cudaStream_t s) {
     e = launch_pdl(topk_hist_kernel, grid, kThreadsTk, 0, s, p);
     if (e != cudaSuccess) return e;
   }
-  e = regs ? launch_pdl(topk_select_kernel<true>, grid, kThreadsTk, smem, s, p)
-           : launch_pdl(topk_select_kernel<false>, grid, kThreadsTk, smem, s, p);
+  if (p.cluster)
+    e = launch_pdl_cluster(topk_select_kernel<true>, grid, kThreadsTk, smem, p.n_seg, s, p);
+  else
+    e = regs ? launch_pdl(topk_select_kernel<true>, grid, kThreadsTk, smem, s, p)
+             : launch_pdl(topk_select_kernel<false>, grid, kThreadsTk, smem, s, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
