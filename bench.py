@@ -8,7 +8,8 @@ window selection, and every sparse layer, all through `hs2_block_decode` (C ABI)
 workload is the 128k-context decode batch: 8 sequences with contexts drawn uniformly from
 65,536..131,072 tokens, 32 query heads on one bf16 K/V head, 3 sparse layers, top-1,024 +
 window 128. Its K/V cache (~400 MB) is larger than the 126 MB L2, so no flush is needed
-between steps.
+between steps. Workloads whose cache fits in L2 (the 4k decode, the 32k prefill) time every step
+alone, after a 256 MB write that evicts the cache, and report the back-to-back time as "warm".
 
 Multi-GPU (torchrun): every rank runs its own batch (independent sequences, no exchange);
 `value` is all ranks' tokens over the slowest rank's time (weak scaling).
@@ -96,7 +97,19 @@ def algorithmic_bytes(w) -> dict:
     tk = T * 4 + B * (w.topk + w.window) * 4
     sel = [min(int(t), w.topk + w.window) for t in w.kv_len]
     sp = sum(sel) * 2 * row + q + o + sum(sel) * 4
-    return dict(pass1=p1, pass2=p2, topk=tk, sparse=sp, total=p1 + p2 + tk + w.n_sparse * sp)
+    total = p1 + p2 + tk + w.n_sparse * sp
+    # B_min: the same step if K were read only once (a design that kept the logits would need
+    # no second K read); reported beside the fraction so that it is not flattered
+    return dict(pass1=p1, pass2=p2, topk=tk, sparse=sp, total=total, total_k_once=total - T * row)
+
+
+L2_BYTES = 126 * 1000 * 1000
+
+
+def cache_bytes(w) -> int:
+    """K and V (and their FP8 scales) of the workload's cache."""
+    return int(w.k.nbytes + w.v.nbytes + (w.k_scale.nbytes + w.v_scale.nbytes
+                                          if w.kv_dtype == "fp8" else 0))
 
 
 class ClockSampler:
@@ -425,21 +438,35 @@ def main():
             pg.barrier()
         torch.cuda.synchronize()
 
-    # ---- timed region: K steps back to back, events only at the two ends
+    # ---- timed region: K steps back to back, events only at the two ends. A cache that fits
+    # in L2 would stay there from step to step, so for such workloads every step is timed
+    # alone after a 256 MB write that evicts it (the back-to-back time is reported as "warm").
+    fits_l2 = cache_bytes(w) < L2_BYTES
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if fits_l2 else None
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     n0 = hs2.launch_count()
     with ClockSampler(local) as clk:
+        if fits_l2:
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(a.steps)]
+            for e0, e1 in pairs:
+                flush.zero_()
+                e0.record(stream)
+                step()
+                e1.record(stream)
         t_start.record(stream)
         for _ in range(a.steps):
             step()
         t_end.record(stream)
         torch.cuda.synchronize()
-    launches = hs2.launch_count() - n0
+    launches = (hs2.launch_count() - n0) // (2 if fits_l2 else 1)
     barrier()
     hs2.read_device_status(ws)
-    ms = t_start.elapsed_time(t_end) / a.steps
+    ms_warm = t_start.elapsed_time(t_end) / a.steps
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in pairs) / a.steps if fits_l2 else ms_warm
     ms_max = slowest(ms, pg, dev)
+    ms_warm_max = slowest(ms_warm, pg, dev)
 
     # ---- the same K steps again with an event between consecutive kernels (per-kernel times;
     # the events break the programmatic-launch overlap, so this step time runs a little longer)
@@ -541,13 +568,18 @@ def main():
         "dtype": "bf16" if w.kv_dtype == "bf16" else "fp8-e4m3 (bf16/f16 math)",
         "data": "synthetic",
         "config": dict(config_of(w), parallelism=f"replicas x{world} (independent batches)",
-                       l2="inputs larger than L2 (K/V cache %.0f MB > 126 MB); no flush"
-                          % (w.k.nbytes * 2 / 1e6)),
+                       l2=("K/V cache %.1f MB fits in L2: every timed step follows a 256 MB "
+                           "write that evicts it; warm back-to-back steps: %.4f ms"
+                           % (cache_bytes(w) / 1e6, ms_warm_max)) if fits_l2 else
+                          ("inputs larger than L2 (K/V cache %.0f MB > 126 MB); no flush"
+                           % (cache_bytes(w) / 1e6))),
         "roofline": roofline,
         **extra,
         "block_roofline": {"bytes_per_step": ab["total"],
                            "achieved_gbs": ab["total"] / (ms_max / 1e3) / 1e9,
-                           "frac": ab["total"] / (ms_max / 1e3) / 1e9 / hbm},
+                           "frac": ab["total"] / (ms_max / 1e3) / 1e9 / hbm,
+                           "bytes_min_k_once": ab["total_k_once"],
+                           "frac_min_k_once": ab["total_k_once"] / (ms_max / 1e3) / 1e9 / hbm},
         "ms_per_kernel": per, "ms_per_step_traced": ms_traced,
         "gpu_launches": int(launches),
         "clocks": clk.result(),
