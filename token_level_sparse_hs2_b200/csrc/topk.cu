@@ -17,7 +17,7 @@
 //     to tau are taken (the lowest indices: a radix select on the index); one more ordered
 //     compaction keeps the selected candidates in ascending order, and the window is appended.
 // Long rows are split over several CTAs (segments). Up to 8 segments form a thread-block
-// cluster and segment 0 gathers the runs from the others' shared memory; more segments compact
+// cluster and each stores its run into segment 0's shared memory; more segments compact
 // into a global buffer and record where their run starts, and the last segment to arrive lays
 // the runs out in segment order. Either way one CTA finishes the row. If the compacted set does not fit (many equal scores),
 // the finishing CTA falls back to exact digit passes and an ordered scan over the whole row.
@@ -146,6 +146,29 @@ __device__ __forceinline__ void ordered_append(uint32_t take_bits, TkSmem &sm, i
   __syncthreads();   // sm.scan is reused by the next step
 }
 
+// Writes, in order, the candidates among the first n <= U * kThreadsTk in shared memory (in
+// ascending position order) whose key is above tau, or equal to it with an index <= ithr.
+template <int U>
+__device__ __forceinline__ void keep_ordered(TkSmem &sm, int n, uint32_t tau, int32_t ithr,
+                                             int topk, int32_t *out) {
+  uint32_t take = 0;
+  int32_t ix[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int j = u * kThreadsTk + threadIdx.x;
+    ix[u] = 0;
+    if (j < n) {
+      const uint32_t k = sm.key[j];
+      ix[u] = sm.idx[j];
+      if (k > tau || (k == tau && ix[u] <= ithr)) take |= 1u << u;
+    }
+  }
+  int run = 0;
+  ordered_append<U>(take, sm, run, [&](int slot, int u) {
+    if (slot < topk) out[slot] = ix[u];
+  });
+}
+
 // Exact finish on n <= kCandCap candidates in shared memory, in ascending position order, that
 // contain every candidate with top digit >= B1 (above = how many have top digit > B1). Writes
 // the ascending selection.
@@ -198,24 +221,11 @@ __device__ void finish_from_smem(TkSmem &sm, int n, int B1, uint32_t above, int 
     ithr = (int32_t)iprefix;
   }
   // the candidates are in ascending position order: keep those above the threshold in that
-  // order (16 steps of kThreadsTk cover kCandCap)
+  // order, with as many steps per thread as the candidates need
   static_assert(kCandCap == 16 * kThreadsTk, "one ordered step covers the candidates");
-  uint32_t take = 0;
-  int32_t ix[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int j = u * kThreadsTk + threadIdx.x;
-    ix[u] = 0;
-    if (j < n) {
-      const uint32_t k = sm.key[j];
-      ix[u] = sm.idx[j];
-      if (k > tau || (k == tau && ix[u] <= ithr)) take |= 1u << u;
-    }
-  }
-  int run = 0;
-  ordered_append<16>(take, sm, run, [&](int slot, int u) {
-    if (slot < topk) out[slot] = ix[u];
-  });
+  if (n <= 4 * kThreadsTk) keep_ordered<4>(sm, n, tau, ithr, topk, out);
+  else if (n <= 8 * kThreadsTk) keep_ordered<8>(sm, n, tau, ithr, topk, out);
+  else keep_ordered<16>(sm, n, tau, ithr, topk, out);
 }
 
 // Exact fallback over the whole candidate row in global memory (any number of equal keys):
@@ -339,7 +349,11 @@ __global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(
     }
   }
   if (gh) {
-    for (int t = threadIdx.x; t < kHistBins; t += kThreadsTk) sm.hist[t] = __ldcg(gh + t);
+    uint32_t hv[kHistBins / kThreadsTk];   // all loads in flight before the first store
+#pragma unroll
+    for (int e = 0; e < kHistBins / kThreadsTk; ++e) hv[e] = __ldcg(gh + e * kThreadsTk + threadIdx.x);
+#pragma unroll
+    for (int e = 0; e < kHistBins / kThreadsTk; ++e) sm.hist[e * kThreadsTk + threadIdx.x] = hv[e];
   } else {   // single segment: build it here
     for (int t = threadIdx.x; t < kHistBins; t += kThreadsTk) sm.hist[t] = 0;
     __syncthreads();
@@ -455,37 +469,40 @@ __global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(
   if (P.n_seg == 1) {
     n = n_local;
   } else if (P.cluster) {
-    // the row's segments form one thread-block cluster: segment 0 gathers the others' runs from
-    // their shared memory in segment order (its own run is already in place) and finishes
+    // the row's segments form one thread-block cluster: every segment reads the counts of the
+    // segments before it and stores its run at that offset into segment 0's shared memory
+    // (remote stores, nothing waits on them), then segment 0 finishes with the runs in segment
+    // order (its own is already in place)
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    if (threadIdx.x == 0) sm.last = n_local;          // this segment's count, for rank 0
+    if (threadIdx.x == 0) sm.last = n_local;          // this segment's count
     cluster.sync();
-    n = 0;
-    if (sg == 0) {
-      const int ns = P.n_seg;
-      const int cnt = threadIdx.x < ns ? *cluster.map_shared_rank(&sm.last, (int)threadIdx.x) : 0;
-      int tot;
-      const int pre = block_excl_scan(cnt, sm.warp_sums, &tot);
-      if (threadIdx.x < ns) sm.seg_pre[threadIdx.x] = pre;
-      __syncthreads();
-      n = tot;
-      if (n <= kCandCap) {
-        for (int j = sm.seg_pre[1 < ns ? 1 : 0] + threadIdx.x; j < n; j += kThreadsTk) {
-          int lo = 1, hi = ns - 1;   // the last segment starting at or before j
-          while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (sm.seg_pre[mid] <= j) lo = mid;
-            else hi = mid - 1;
-          }
-          const int off = j - sm.seg_pre[lo];
-          sm.key[j] = cluster.map_shared_rank(sm.key, lo)[off];
-          sm.idx[j] = cluster.map_shared_rank(sm.idx, lo)[off];
-        }
+    const int ns = P.n_seg;
+    int cnt = (threadIdx.x < 32 && (int)threadIdx.x < ns) ? *cluster.map_shared_rank(&sm.last, (int)threadIdx.x) : 0;
+    int pre = (threadIdx.x < 32 && (int)threadIdx.x < sg) ? cnt : 0;
+    if (threadIdx.x < 32) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        pre += __shfl_xor_sync(0xffffffffu, pre, o);
       }
-      __syncthreads();
+      if (threadIdx.x == 0) {
+        sm.seg_pre[0] = pre;   // this segment's offset in segment 0's buffer
+        sm.seg_pre[1] = cnt;   // the row's candidates
+      }
     }
-    cluster.sync();   // no segment leaves while rank 0 may still read its shared memory
+    __syncthreads();
+    pre = sm.seg_pre[0];
+    n = sm.seg_pre[1];
+    if (sg != 0 && n <= kCandCap) {
+      uint32_t *rkey = cluster.map_shared_rank(sm.key, 0);
+      int32_t *ridx = cluster.map_shared_rank(sm.idx, 0);
+      for (int j = threadIdx.x; j < n_local; j += kThreadsTk) {
+        rkey[pre + j] = sm.key[j];
+        ridx[pre + j] = sm.idx[j];
+      }
+    }
+    cluster.sync();   // the runs are in segment 0's shared memory (release / acquire)
     if (sg != 0) return;
   } else {
     // publish this segment's candidates with one global reservation and record where they
