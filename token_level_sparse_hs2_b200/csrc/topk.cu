@@ -123,25 +123,29 @@ __device__ __forceinline__ uint32_t load_key(const float *s, int64_t t) {
 // U x kWarpsTk counts give every element its slot.
 template <int U, class Emit>
 __device__ __forceinline__ void ordered_append(uint32_t take_bits, TkSmem &sm, int &run, Emit emit) {
-  static_assert(U * kWarpsTk <= kThreadsTk, "one scan entry per thread");
+  static_assert(U * kWarpsTk <= kThreadsTk && U <= 32, "one scan entry per thread");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned m[U];
+  int mine = 0;   // lane u holds the count of step u
 #pragma unroll
-  for (int u = 0; u < U; ++u) m[u] = __ballot_sync(0xffffffffu, (take_bits >> u) & 1u);
-  if (lane == 0) {
-#pragma unroll
-    for (int u = 0; u < U; ++u) sm.scan[u * kWarpsTk + warp] = __popc(m[u]);
+  for (int u = 0; u < U; ++u) {
+    m[u] = __ballot_sync(0xffffffffu, (take_bits >> u) & 1u);
+    if (lane == u) mine = __popc(m[u]);
   }
+  if (lane < U) sm.scan[lane * kWarpsTk + warp] = mine;
   __syncthreads();
   const int v = threadIdx.x < U * kWarpsTk ? sm.scan[threadIdx.x] : 0;
   int tot;
   const int ex = block_excl_scan(v, sm.warp_sums, &tot);
   if (threadIdx.x < U * kWarpsTk) sm.scan[threadIdx.x] = ex;
   __syncthreads();
+  const int base_mine = lane < U ? sm.scan[lane * kWarpsTk + warp] : 0;   // offset of step lane
   const unsigned below = (1u << lane) - 1u;
 #pragma unroll
-  for (int u = 0; u < U; ++u)
-    if ((take_bits >> u) & 1u) emit(run + sm.scan[u * kWarpsTk + warp] + __popc(m[u] & below), u);
+  for (int u = 0; u < U; ++u) {
+    const int base = __shfl_sync(0xffffffffu, base_mine, u);
+    if ((take_bits >> u) & 1u) emit(run + base + __popc(m[u] & below), u);
+  }
   run += tot;
   __syncthreads();   // sm.scan is reused by the next step
 }
