@@ -1,6 +1,7 @@
-"""The context-parallel decode orchestration on CPU: world size 2 over gloo (127.0.0.1).
+"""The context-parallel decode orchestration on CPU: world sizes 2 and 3 over gloo (127.0.0.1).
 
-cp_block_decode is run unchanged by two processes, each holding one token range of a sequence,
+cp_block_decode is run unchanged by two or three processes, each holding one token range of a
+sequence (one case puts a whole shard inside the forced window, so it offers no candidates),
 with its collectives over gloo and its per-shard operations replaced by a float64 CPU stand-in
 written here (the oracle's attention and selection on the shard, numpy merges). The merged
 results must equal the oracle's single-process block over the whole context: full-layer output
@@ -159,12 +160,13 @@ def _rank(rank, world, port, bounds, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("bounds", [[0, 350, 700], [0, 650, 700]])
-def test_two_rank_cp_decode_equals_the_whole_context(oracle_lib, bounds):
+@pytest.mark.parametrize("bounds", [[0, 350, 700], [0, 650, 700], [0, 400, 690, 700]])
+def test_cp_decode_over_gloo_equals_the_whole_context(oracle_lib, bounds):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29700 + os.getpid() % 1000 + bounds[1] % 97
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, bounds, q)) for r in range(2)]
+    world = len(bounds) - 1
+    port = 29700 + os.getpid() % 1000 + bounds[1] % 97 + 101 * (world - 2)
+    procs = [ctx.Process(target=_rank, args=(r, world, port, bounds, q)) for r in range(world)]
     for p in procs:
         p.start()
     got = []
