@@ -220,3 +220,61 @@ def test_context_parallel_argument_checks(L):
                                  1152, P(256), None) == 2          # 32 x 1024 keys: too many
     assert L.hs2_cp_localize(1, (ctypes.c_int64 * 1)(4000), (ctypes.c_int32 * 1)(1000), P(256),
                              1152, P(256), P(256), 100, P(256), None) == 1
+
+
+def declared_signatures():
+    """name -> (return type, [parameter types]) of every function include/*.h declares."""
+    sigs = {}
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"#[^\n]*", "", src)
+        for m in re.finditer(r"([A-Za-z_][A-Za-z0-9_ ]*?[\s\*]+)(hs2_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src):
+            ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+            if params in ("", "void"):
+                sigs[name] = (ret, [])
+                continue
+            types = []
+            for p in params.split(","):
+                p = " ".join(p.split())
+                # drop the parameter name (the last identifier) unless the parameter is unnamed
+                t = re.sub(r"\s*\b[A-Za-z_][A-Za-z0-9_]*$", "", p) if not p.endswith("*") else p
+                types.append(t if t else p)
+            sigs[name] = (ret, types)
+    return sigs
+
+
+def ctype_class(t: str) -> str:
+    t = t.replace("const", "").strip()
+    if "*" in t:
+        return "pointer"
+    return {"int32_t": "i32", "int64_t": "i64", "uint32_t": "u32", "uint64_t": "u64",
+            "size_t": "size", "float": "f32", "int": "i32", "hs2_status": "i32"}.get(t, t)
+
+
+def argtype_class(a) -> str:
+    if a in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(a, "_type_") and \
+            isinstance(getattr(a, "_type_", None), type):
+        return "pointer"
+    return {ctypes.c_int32: "i32", ctypes.c_int64: "i64", ctypes.c_uint32: "u32",
+            ctypes.c_uint64: "u64", ctypes.c_size_t: "size", ctypes.c_float: "f32"}.get(a, repr(a))
+
+
+def test_binding_argtypes_match_the_header(L):
+    """Every argument list the binding declares has the header's length and, argument by
+    argument, the same class (pointer, 32/64-bit integer, size_t, float)."""
+    sigs = declared_signatures()
+    assert "hs2_block_decode" in sigs and len(sigs["hs2_block_decode"][1]) == 19
+    checked = 0
+    for name, (ret, params) in sorted(sigs.items()):
+        fn = getattr(L, name)
+        if fn.argtypes is None:
+            assert not params, f"{name}: the binding sets no argument types"
+            continue
+        got = [argtype_class(a) for a in fn.argtypes]
+        want = [ctype_class(p) for p in params]
+        assert got == want, (name, got, want)
+        checked += 1
+    assert checked >= 20
