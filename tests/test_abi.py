@@ -278,3 +278,48 @@ def test_binding_argtypes_match_the_header(L):
         assert got == want, (name, got, want)
         checked += 1
     assert checked >= 20
+
+
+def test_view_struct_matches_the_header():
+    """The binding's hs2_kv_view has the header's fields in the header's order, with the same
+    widths, so every offset agrees (the library reads the struct by those offsets)."""
+    src = open(os.path.join(ROOT, "include", "hs2.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    body = re.search(r"typedef struct hs2_kv_view \{(.*?)\} hs2_kv_view;", src, flags=re.S).group(1)
+    fields = []
+    for decl in body.split(";"):
+        decl = " ".join(decl.split())
+        if not decl:
+            continue
+        name = re.search(r"([A-Za-z_][A-Za-z0-9_]*)$", decl).group(1)
+        fields.append((name, ctype_class(decl[: -len(name)].strip())))
+    got = [(n, argtype_class(t)) for n, t in hs2._KvView._fields_]
+    assert got == fields
+    offsets, off = [], 0
+    for _, cls in fields:   # natural alignment on a 64-bit host
+        size = {"i32": 4, "u32": 4, "f32": 4}.get(cls, 8)
+        off = (off + size - 1) // size * size
+        offsets.append(off)
+        off += size
+    assert [getattr(hs2._KvView, n).offset for n, _ in hs2._KvView._fields_] == offsets
+    assert ctypes.sizeof(hs2._KvView) == (off + 7) // 8 * 8
+
+
+def test_view_layout_agrees_with_the_c_compiler(tmp_path):
+    """The header compiles as plain C (C99, no CUDA headers), and gcc lays hs2_kv_view out at
+    the offsets the binding uses."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc is not installed")
+    names = [n for n, _ in hs2._KvView._fields_]
+    prints = "".join(f'printf("%zu\\n", offsetof(hs2_kv_view, {n}));' for n in names)
+    (tmp_path / "lay.c").write_text(
+        "#include <stdio.h>\n#include <stddef.h>\n#include \"hs2.h\"\n"
+        f"int main(void){{{prints} printf(\"%zu\\n\", sizeof(hs2_kv_view)); return 0;}}\n")
+    exe = tmp_path / "lay"
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I" + os.path.join(ROOT, "include"),
+                           str(tmp_path / "lay.c"), "-o", str(exe)])
+    out = [int(x) for x in subprocess.check_output([str(exe)]).split()]
+    assert out[:-1] == [getattr(hs2._KvView, n).offset for n in names]
+    assert out[-1] == ctypes.sizeof(hs2._KvView)
