@@ -86,11 +86,18 @@ typedef struct hs2_kv_view {
   const int32_t *kv_len;     /* HOST [batch], T_b */
 } hs2_kv_view;
 
+/* Outputs of hs2_block_decode that the caller may leave to the library (pass NULL for them): the
+ * flags of hs2_workspace_size that reserve room for them in the workspace. */
+#define HS2_WS_SCORES 1u      /* scores == NULL: the [B*Nq, max p + 1] fp32 scores */
+#define HS2_WS_SELECTION 2u   /* idx == count == NULL: the selected positions and their counts */
+
 /* Bytes of device scratch the calls below need for this view and budget (same value for every
- * call on the view). Any 256-byte-aligned device buffer of at least this size works; its
- * contents on entry do not matter. Host-only; does not touch the GPU. */
+ * call on the view). flags: 0, or HS2_WS_SCORES and / or HS2_WS_SELECTION for an
+ * hs2_block_decode call that leaves those outputs to the workspace. Any 256-byte-aligned device
+ * buffer of at least this size works; its contents on entry do not matter. Host-only; does not
+ * touch the GPU. Unknown flag bits: HS2_ERR_INVALID_ARG. */
 hs2_status hs2_workspace_size(const hs2_kv_view *kv, int32_t topk, int32_t window,
-                              size_t *bytes);
+                              uint32_t flags, size_t *bytes);
 
 /* Step 1 -- the full-attention layer and its importance scores (pages: section "KV Reuse and
  * Token-Level Sparse Selection"; the full layer attends causally over the entire context).
@@ -112,7 +119,9 @@ hs2_status hs2_full_attn_scores(const hs2_kv_view *kv, const void *q, float soft
  * is [0, p]; otherwise it is the topk candidates with the largest score (ties: lower index),
  * followed by W, all ascending. Scores are compared by their fp32 bit patterns, which for the
  * non-negative scores step 1 produces is the numeric order (an exact, deterministic radix
- * select). idx: device int32 [B*Nq, idx_stride], idx_stride >= min(max p + 1, topk + window);
+ * select). A candidate score that is negative (-0.0 included) or NaN breaks that order: the
+ * call still completes and records HS2_ERR_DEVICE_CHECK in the device status.
+ * idx: device int32 [B*Nq, idx_stride], idx_stride >= min(max p + 1, topk + window);
  * only the first count[r] entries of row r are written. count: device int32 [B*Nq]. */
 hs2_status hs2_topk_select(const hs2_kv_view *kv, const float *scores, int64_t score_stride,
                            int32_t topk, int32_t window, int32_t *idx, int32_t idx_stride,
@@ -134,7 +143,10 @@ hs2_status hs2_sparse_gather_attn(const hs2_kv_view *kv, const void *q, const in
 /* The whole hybrid block: step 1, step 2, then n_sparse sparse layers that reuse the indices
  * and the cache, enqueued back to back on `stream`. q_sparse / out_sparse are HOST arrays of
  * n_sparse device pointers (layouts as in step 3). lse, scores, idx and count are outputs too
- * (caller-provided, layouts as above). n_sparse may be 0. */
+ * (layouts as above), each optional: a NULL lse, a NULL scores (score_stride is then ignored) or
+ * NULL idx and count (idx_stride ignored; both or neither) are kept in the workspace instead,
+ * which must then hold hs2_workspace_size(kv, topk, window, flags) bytes with HS2_WS_SCORES /
+ * HS2_WS_SELECTION set for the NULL ones (the lse always fits). n_sparse may be 0. */
 hs2_status hs2_block_decode(const hs2_kv_view *kv, const void *q_full,
                             const void *const *q_sparse, int32_t n_sparse, int32_t topk,
                             int32_t window, float softmax_scale, void *out_full,
@@ -175,12 +187,20 @@ hs2_status hs2_block_decode_traced(const hs2_kv_view *kv, const void *q_full,
  *    start at zero are cleared on the stream at the start of each call). Calls that can
  *    overlap on the GPU -- on different streams, or from different host threads -- race on it
  *    and must be serialised by the caller.
- *  - Errors the kernels detect themselves are recorded in the shared array and are not
- *    reported by hs2_read_device_status. */
+ *  - The one error the selection kernels detect themselves (a negative or NaN candidate score,
+ *    see hs2_topk_select; the selection has no waits that could run out) goes to a status word
+ *    in the array: read it with hs2_noalloc_read_status (hs2_read_device_status needs a
+ *    workspace). Each call clears it when it starts. */
 hs2_status hs2_topk_select_noalloc(const hs2_kv_view *kv, const float *scores,
                                    int64_t score_stride, int32_t topk, int32_t window,
                                    int32_t *idx, int32_t idx_stride, int32_t *count,
                                    void *stream);
+
+/* Synchronises `stream`, then returns the status the last hs2_topk_select_noalloc call on the
+ * current device recorded in the built-in array (HS2_OK, or HS2_ERR_DEVICE_CHECK for a negative
+ * or NaN candidate score) and clears it. HS2_ERR_CUDA if the read fails. Like the selection, it
+ * calls no allocator; it races with a selection still running on another stream. */
+hs2_status hs2_noalloc_read_status(void *stream);
 
 /* Block-level variant of step 2: the granularity HySparse used and HySparse2 replaces
  * ("HySparse2: How Xiaomi Split the Transformer to Fix Agent Prefill Costs", section "KV Reuse and
@@ -221,8 +241,8 @@ int32_t hs2_version(void);
  * already counts) receives new_k[b][i][:] and new_v[b][i][:] (device, bf16 [batch, n_q, 128],
  * 16-byte aligned). bf16 cache: copied. e4m3 cache: per row and matrix, scale = max|x| / 448 in
  * float32 (1 for an all-zero row) is written to k_scale / v_scale and the codes are the
- * round-to-nearest-even e4m3 of x * (1 / scale) (the reciprocal rounded to float32), saturated
- * at 448. The view's K/V (and scale) buffers
+ * round-to-nearest-even e4m3 of the float32 quotient x / scale (IEEE division, correctly
+ * rounded), saturated at 448. The view's K/V (and scale) buffers
  * are written: they are caller-owned device memory. Asynchronous on `stream`; argument errors
  * return before any launch. */
 hs2_status hs2_kv_append(const hs2_kv_view *kv, const void *new_k, const void *new_v, void *stream);

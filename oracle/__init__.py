@@ -290,7 +290,7 @@ def e4m3_rne(y: float) -> int:
 
 def quantize_rows(x_bf16_bits: np.ndarray):
     """FP8 cache rows for appended tokens: x as bf16 bits [rows, d] -> (codes uint8 [rows, d],
-    scale float32 [rows]); scale = max|x| / 448 (1 for a zero row), codes = e4m3 RNE of x * (1 / scale)."""
+    scale float32 [rows]); scale = max|x| / 448 (1 for a zero row), codes = e4m3 RNE of the float32 quotient x / scale."""
     x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
     rows, d = x.shape
     codes = np.zeros((rows, d), dtype=np.uint8)

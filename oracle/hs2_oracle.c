@@ -511,9 +511,10 @@ uint8_t hs2o_e4m3_rne(float y) {
   return (uint8_t)(code | (neg << 7));
 }
 
-/* The FP8 cache write of one appended row of d bf16 values: scale = max|x| / 448 in float32
- * (1 for an all-zero row), codes = e4m3 RNE of the float32 product x * r, r = 1 / scale rounded
- * to float32, saturated at 448. */
+/* The FP8 cache write of one appended row of d bf16 values, from the format's definition
+ * value = scale * code: scale = max|x| / 448 in float32 (1 for an all-zero row), and each code is
+ * the e4m3 RNE of the float32 quotient x / scale (IEEE division, correctly rounded), saturated
+ * at 448. */
 void hs2o_quantize_row(const uint16_t *x_bf16, int d, uint8_t *codes, float *scale) {
   float amax = 0.f;
   for (int j = 0; j < d; ++j) {
@@ -523,12 +524,11 @@ void hs2o_quantize_row(const uint16_t *x_bf16, int d, uint8_t *codes, float *sca
     if (fabsf(v) > amax) amax = fabsf(v);
   }
   const float sc = amax > 0.f ? amax / 448.0f : 1.0f;
-  const float r = 1.0f / sc;
   for (int j = 0; j < d; ++j) {
     uint32_t u = (uint32_t)x_bf16[j] << 16;
     float v;
     memcpy(&v, &u, 4);
-    const float y = v * r;
+    const float y = v / sc;
     codes[j] = hs2o_e4m3_rne(y);
   }
   *scale = sc;

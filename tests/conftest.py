@@ -11,6 +11,8 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size oracle comparison")
+    config.addinivalue_line("markers", "fullparity: every query row of a full-size workload "
+                            "against the oracle (needs a CUDA device; minutes of host time)")
 
 
 @pytest.fixture(scope="session")

@@ -149,6 +149,43 @@ def test_call_argument_checks_before_any_launch(L):
     assert st == 1 and b"score_stride" in hs2.lib().hs2_last_error()
 
 
+def test_optional_block_outputs_sizes_and_checks(L):
+    """scores / idx + count may be NULL in hs2_block_decode: hs2_workspace_size's flags reserve
+    room for them (scores: rows x (max p + 1, rounded up to 64) floats; selection: rows x
+    min(max p + 1, topk + window) positions plus the counts), and a call that leaves an output
+    to a workspace sized without its flag is refused on the host before any launch."""
+    c = cpu_cache(lens=(300, 500))
+    base = hs2.workspace_size(c)
+    with_scores = hs2.workspace_size(c, flags=hs2.WS_SCORES)
+    with_sel = hs2.workspace_size(c, flags=hs2.WS_SELECTION)
+    both = hs2.workspace_size(c, flags=hs2.WS_SCORES | hs2.WS_SELECTION)
+    assert with_scores - base >= 2 * 512 * 4
+    assert with_sel - base >= 2 * 500 * 4 + 2 * 4
+    assert both - base >= (with_scores - base) + (with_sel - base) - 512
+    assert status_of(lambda: hs2.workspace_size(c, flags=4))[0] == 1
+    H = 32
+    q = torch.zeros((2, 1, H, 128), dtype=torch.bfloat16)
+    out = torch.zeros_like(q, dtype=torch.float32)
+    idx = torch.zeros((2, 500), dtype=torch.int32)
+    cnt = torch.zeros(2, dtype=torch.int32)
+    buf = torch.zeros(both + 256, dtype=torch.uint8)
+    ws = buf.data_ptr() + (-buf.data_ptr()) % 256
+    raw = hs2.lib().hs2_block_decode
+    def call(scores_p, idx_p, cnt_p, ws_bytes):
+        return raw(c.ref(), q.data_ptr(), (ctypes.c_void_p * 1)(q.data_ptr()), 1, 1024, 128,
+                   0.088, out.data_ptr(), (ctypes.c_void_p * 1)(out.data_ptr()), 1, None,
+                   scores_p, 0, idx_p, 0, cnt_p, ws, ws_bytes, None)
+    # idx without count (or the reverse) is an argument error
+    assert call(None, idx.data_ptr(), None, both) == 1
+    assert b"both" in hs2.lib().hs2_last_error()
+    assert call(None, None, cnt.data_ptr(), both) == 1
+    # NULL outputs with a workspace sized for fewer of them: refused with the size
+    assert call(None, None, None, with_scores) == 3
+    assert call(None, None, None, with_sel) == 3
+    assert call(None, idx.data_ptr(), cnt.data_ptr(), base) == 3
+    assert b"required" in hs2.lib().hs2_last_error()
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     import importlib
     mod = importlib.import_module("token_level_sparse_hs2_b200")
@@ -165,9 +202,12 @@ def test_noalloc_selection_rejects_oversized_calls(L):
     scores = torch.zeros((100, 20000))
     idx = torch.zeros((100, 1152), dtype=torch.int32)
     cnt = torch.zeros(100, dtype=torch.int32)
+    idx.fill_(-7)
+    cnt.fill_(-7)
     st = hs2.lib().hs2_topk_select_noalloc(c.ref(), scores.data_ptr(), 20000, 1024, 128,
                                            idx.data_ptr(), 1152, cnt.data_ptr(), None)
     assert st == 3 and b"scratch" in hs2.lib().hs2_last_error()
+    assert (idx == -7).all() and (cnt == -7).all()   # refused before anything was written
 
 
 def test_selftest_rejects_bad_arguments_without_launching():

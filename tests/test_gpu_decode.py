@@ -235,3 +235,31 @@ def test_scattered_sequences_and_custom_scale(kv_dtype):
     w = scatter(base, 6)
     g = H().run_block(w, scale=0.05)
     H().check_block(w, g, scale=0.05)
+
+
+@pytest.mark.parametrize("kv_dtype,n_q", [("bf16", 1), ("fp8", 1), ("bf16", 40)])
+def test_optional_outputs_left_to_the_workspace(kv_dtype, n_q):
+    """hs2_block_decode with NULL lse, scores, idx and count (the library keeps them in the
+    workspace): the block outputs equal, bit for bit, those of the same call with every output
+    given, and that call matches the oracle."""
+    import token_level_sparse_hs2_b200 as hs2
+    w = decode(batch=3, n_q=n_q, lengths=(5000, 2100, 3333), kv_dtype=kv_dtype, needles=3,
+               n_heads=32, n_sparse=2)
+    g = H().run_block(w)
+    H().check_block(w, g)
+    cache, d = g["cache"], g["dev"]
+    dev = d["k"].device
+    out_full = torch.empty((w.batch, w.n_q, w.n_heads, 128), dtype=torch.float32, device=dev)
+    out_sp = [torch.empty_like(out_full) for _ in range(w.n_sparse)]
+    nbytes = hs2.workspace_size(cache, flags=hs2.WS_SCORES | hs2.WS_SELECTION)
+    assert nbytes > hs2.workspace_size(cache)
+    ws = torch.full((nbytes,), 0xff, dtype=torch.uint8, device=dev)
+    for _ in range(2):   # twice: the workspace's previous contents must not matter
+        hs2.block_decode(cache, d["q_full"], d["q_sparse"], out_full, out_sp, None, None, None,
+                         None, ws)
+        hs2.read_device_status(ws)
+        R = w.n_rows
+        np.testing.assert_array_equal(out_full.reshape(R, w.n_heads, 128).cpu().numpy(), g["o_full"])
+        for l in range(w.n_sparse):
+            np.testing.assert_array_equal(out_sp[l].reshape(R, w.n_heads, 128).cpu().numpy(),
+                                          g["o_sparse"][l])

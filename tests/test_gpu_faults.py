@@ -57,3 +57,26 @@ def test_count_out_of_range_is_clamped_and_reported():
     with pytest.raises(hs2.HS2Error) as e:
         hs2.read_device_status(ws)
     assert e.value.status == HS2_ERR_DEVICE_CHECK
+
+
+def test_negative_or_nan_scores_are_reported_by_the_selection():
+    """hs2_topk_select on caller scores that break the non-negative order: the call completes
+    and the device status reports a check, for a split row and for many unsplit rows."""
+    dev = torch.device("cuda")
+    for lens, bad in (((50000,), float("nan")), ((3000,) * 150, -0.0)):
+        w = W.make_workload(dict(name="negscore", batch=len(lens), n_q=1, n_heads=16, n_sparse=0,
+                                 kv_dtype="bf16", lengths=lens, needles=0), seed=9)
+        d = W.to_device(w, dev)
+        cache = hs2.KvCache(d["k"], d["v"], w.kv_start, w.kv_len, 1, w.n_heads)
+        s = torch.rand((len(lens), max(lens)), device=dev)
+        s[-1, 1000] = bad
+        idx = torch.empty((len(lens), 1152), dtype=torch.int32, device=dev)
+        cnt = torch.empty(len(lens), dtype=torch.int32, device=dev)
+        ws = torch.empty(hs2.workspace_size(cache), dtype=torch.uint8, device=dev)
+        hs2.topk_select(cache, s, idx, cnt, ws)
+        with pytest.raises(hs2.HS2Error) as e:
+            hs2.read_device_status(ws)
+        assert e.value.status == HS2_ERR_DEVICE_CHECK
+        s[-1, 1000] = 0.5
+        hs2.topk_select(cache, s, idx, cnt, ws)
+        hs2.read_device_status(ws)

@@ -77,7 +77,8 @@ def test_config3_chunk_full_size():
 @pytest.mark.slow
 def test_config4_prefill_full_size():
     w = W.make_workload(4)
-    rows = W.sample_rows(w, 48, extra=(0, 127, 128, 1150, 1151, 1152, 1153, 32767))
+    rows = W.sample_rows(w, 320, extra=(0, 1, 126, 127, 128, 129, 1150, 1151, 1152, 1153, 1154,
+                                        16383, 16384, 32766, 32767))
     g = H().run_block(w, rows=rows)
     H().check_block(w, g)
     for j, r in enumerate(rows):

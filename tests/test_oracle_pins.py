@@ -316,6 +316,56 @@ def test_quantize_rows_scale_codes_and_error_bound(oracle_lib):
     assert codes[5, 17] == 0xfe and np.all(codes[5, np.arange(128) != 17] == 0)
 
 
+def _e4m3_by_torch(y: np.ndarray) -> np.ndarray:
+    """torch's float8_e4m3fn cast (round to nearest even) of float32 values clamped to +-448."""
+    y = np.clip(y.astype(np.float32), -448.0, 448.0)
+    return torch.from_numpy(np.ascontiguousarray(y)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_quantize_rows_codes_are_the_rounded_quotient(oracle_lib):
+    """The codes follow value = scale * code: each is the e4m3 rounding of the float32 quotient
+    x / scale (numpy's IEEE float32 division), cast by torch -- an implementation independent of
+    the oracle's own e4m3 encoder -- on 4,096 random rows whose magnitudes span 2^-20 .. 2^20."""
+    rng = np.random.default_rng(81)
+    rows = 4096
+    mag = np.exp2(rng.uniform(-20, 20, (rows, 1))).astype(np.float32)
+    x = rng.standard_normal((rows, 128)).astype(np.float32) * mag
+    x[::97] *= rng.uniform(0.0, 1e-3, (x[::97].shape[0], 128)).astype(np.float32)  # tiny tails
+    bits = W.f32_to_bf16_bits(x)
+    xf = W.bf16_bits_to_f32(bits)
+    codes, scale = oracle_lib.quantize_rows(bits)
+    amax = np.abs(xf).max(axis=1)
+    want_scale = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+    np.testing.assert_array_equal(scale, want_scale)
+    quotient = (xf / want_scale[:, None]).astype(np.float32)
+    np.testing.assert_array_equal(codes, _e4m3_by_torch(quotient))
+
+
+def test_quantize_rows_rejects_the_reciprocal_product(oracle_lib):
+    """x * rn(1/scale) and rn(x / scale) straddle an e4m3 rounding boundary for some inputs; on
+    exactly those the oracle must give the quotient's code (a planted reciprocal form fails)."""
+    rng = np.random.default_rng(82)
+    found = 0
+    for _ in range(64):
+        x = (rng.standard_normal((512, 128)) * np.exp2(rng.uniform(-8, 8, (512, 1)))).astype(np.float32)
+        bits = W.f32_to_bf16_bits(x)
+        xf = W.bf16_bits_to_f32(bits)
+        amax = np.abs(xf).max(axis=1)
+        sc = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+        q_code = _e4m3_by_torch(xf / sc[:, None])
+        r_code = _e4m3_by_torch(xf * (np.float32(1.0) / sc)[:, None])
+        rows = np.nonzero((q_code != r_code).any(axis=1))[0]
+        if rows.size == 0:
+            continue
+        codes, _ = oracle_lib.quantize_rows(bits[rows])
+        np.testing.assert_array_equal(codes, q_code[rows])
+        assert (codes != r_code[rows]).any()
+        found += rows.size
+        if found >= 8:
+            break
+    assert found >= 8, "no straddling inputs found"
+
+
 # ------------------------------------------------------------------ KV Bridging projections
 
 def test_kv_bridge_equals_float64_matmul(oracle_lib):

@@ -3,15 +3,18 @@
 latency-critical path that must not call cudaMalloc) -- checked through the C ABI against
 hs2_topk_select with a caller workspace. Selection is integer work, so the two must agree
 exactly, on two calls in a row (the built-in scratch keeps the previous call's contents).
-This file is collected last on purpose."""
+Every way the selection splits its rows is covered: a few rows over a cluster of segments, one
+row over more segments than a cluster holds (candidates through the scratch's global buffers),
+and many rows of one CTA each. This file is collected last on purpose."""
 import numpy as np
 import pytest
 import torch
 
 import token_level_sparse_hs2_b200 as hs2
-import workloads as W
 
 pytestmark = pytest.mark.gpu
+
+HS2_ERR_WORKSPACE, HS2_ERR_DEVICE_CHECK = 3, 5
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -30,26 +33,81 @@ def scores_for(lens, seed, quant):
     return s
 
 
-def test_noalloc_selection_matches_workspace_selection():
-    lens = (100000, 60003, 4000)
-    w = W.make_workload(dict(name="noalloc", batch=3, n_q=1, n_heads=32, n_sparse=0,
-                             kv_dtype="bf16", lengths=lens, needles=0), seed=3)
-    d = W.to_device(w)
-    cache = hs2.KvCache(d["k"], d["v"], w.kv_start, w.kv_len, 1, w.n_heads)
-    dev = d["k"].device
+def cache_for(lens):
+    # the selection reads only the scores and the sequence geometry: every sequence views the
+    # same rows of one small cache (rows [0, T_b)), which the view allows
+    dev = torch.device("cuda")
+    k = torch.zeros((max(lens), 128), dtype=torch.bfloat16, device=dev)
+    return hs2.KvCache(k, k, [0] * len(lens), lens, 1, 32), dev
+
+
+def compare_twice(lens, draws):
+    cache, dev = cache_for(lens)
+    B = len(lens)
     ws = torch.empty(hs2.workspace_size(cache), dtype=torch.uint8, device=dev)
-    for call, (seed, quant) in enumerate([(11, 0), (12, 8)]):
+    for call, (seed, quant) in enumerate(draws):
         s = torch.from_numpy(scores_for(lens, seed, quant)).to(dev)
-        idx_a = torch.full((3, 1152), -1, dtype=torch.int32, device=dev)
-        cnt_a = torch.zeros(3, dtype=torch.int32, device=dev)
-        idx_b = torch.full((3, 1152), -2, dtype=torch.int32, device=dev)
-        cnt_b = torch.full((3,), -1, dtype=torch.int32, device=dev)
+        idx_a = torch.full((B, 1152), -1, dtype=torch.int32, device=dev)
+        cnt_a = torch.zeros(B, dtype=torch.int32, device=dev)
+        idx_b = torch.full((B, 1152), -2, dtype=torch.int32, device=dev)
+        cnt_b = torch.full((B,), -1, dtype=torch.int32, device=dev)
         hs2.topk_select(cache, s, idx_a, cnt_a, ws)
         hs2.read_device_status(ws)
         hs2.topk_select_noalloc(cache, s, idx_b, cnt_b)
-        torch.cuda.synchronize()
+        hs2.noalloc_read_status()
         ca, cb = cnt_a.cpu().numpy(), cnt_b.cpu().numpy()
         assert np.array_equal(ca, cb), (call, ca, cb)
         ia, ib = idx_a.cpu().numpy(), idx_b.cpu().numpy()
-        for r in range(3):
+        for r in range(B):
             assert np.array_equal(ia[r, :ca[r]], ib[r, :cb[r]]), (call, r)
+
+
+def test_noalloc_selection_matches_workspace_selection():
+    # three rows, each split over at most 7 segments of one thread-block cluster
+    compare_twice((100000, 60003, 4000), [(11, 0), (12, 8)])
+
+
+def test_noalloc_selection_over_many_segments():
+    # one row of about 300k positions: 19 segments, more than a cluster holds, so the
+    # candidates go through the scratch's global buffers and arrival counters, which the
+    # second call must find reset
+    compare_twice((300007,), [(21, 0), (22, 4)])
+
+
+def test_noalloc_selection_many_rows():
+    # 160 rows: one CTA per row, no split
+    rng = np.random.default_rng(5)
+    lens = tuple(int(x) for x in rng.integers(900, 5000, size=160))
+    compare_twice(lens, [(31, 0), (32, 16)])
+
+
+def test_noalloc_rejects_a_plan_above_the_builtin_scratch():
+    # 60 rows of 200,000 positions split over many segments need more than 4 MiB: refused on
+    # the host with the workspace status, nothing launched, the outputs left as they were
+    lens = (200000,) * 60
+    cache, dev = cache_for(lens)
+    s = torch.zeros((60, 200000), dtype=torch.float32, device=dev)
+    idx = torch.full((60, 1152), -7, dtype=torch.int32, device=dev)
+    cnt = torch.full((60,), -7, dtype=torch.int32, device=dev)
+    with pytest.raises(hs2.HS2Error) as e:
+        hs2.topk_select_noalloc(cache, s, idx, cnt)
+    assert e.value.status == HS2_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert (idx == -7).all() and (cnt == -7).all()
+
+
+def test_noalloc_reports_a_negative_score_and_clears_it():
+    lens = (100000, 4000)
+    cache, dev = cache_for(lens)
+    s = torch.from_numpy(scores_for(lens, 41, 0)).to(dev)
+    s[0, 777] = -1.0          # breaks the bit-pattern order the radix select relies on
+    idx = torch.empty((2, 1152), dtype=torch.int32, device=dev)
+    cnt = torch.empty(2, dtype=torch.int32, device=dev)
+    hs2.topk_select_noalloc(cache, s, idx, cnt)
+    with pytest.raises(hs2.HS2Error) as e:
+        hs2.noalloc_read_status()
+    assert e.value.status == HS2_ERR_DEVICE_CHECK
+    hs2.noalloc_read_status()   # the read cleared it
+    s[0, 777] = 1.0
+    hs2.topk_select_noalloc(cache, s, idx, cnt)
+    hs2.noalloc_read_status()   # a clean call reports nothing

@@ -23,7 +23,7 @@ from typing import Optional, Sequence
 
 import torch
 
-__all__ = ["HS2Error", "KvCache", "lib", "workspace_size", "full_attn_scores", "topk_select",
+__all__ = ["HS2Error", "KvCache", "lib", "workspace_size", "WS_SCORES", "WS_SELECTION", "full_attn_scores", "topk_select",
            "sparse_gather_attn", "block_decode", "read_device_status", "default_scale",
            "KV_BF16", "KV_FP8_E4M3", "OUT_BF16", "OUT_F32", "TOPK", "WINDOW"]
 
@@ -70,7 +70,7 @@ def lib() -> ctypes.CDLL:
         P, I32, I64, F, SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
                               ctypes.c_size_t)
         V = ctypes.POINTER(_KvView)
-        L.hs2_workspace_size.argtypes = [V, I32, I32, ctypes.POINTER(SZ)]
+        L.hs2_workspace_size.argtypes = [V, I32, I32, ctypes.c_uint32, ctypes.POINTER(SZ)]
         L.hs2_full_attn_scores.argtypes = [V, P, F, P, I32, P, P, I64, P, SZ, P]
         L.hs2_topk_select.argtypes = [V, P, I64, I32, I32, P, I32, P, P, SZ, P]
         L.hs2_sparse_gather_attn.argtypes = [V, P, P, I32, P, F, P, I32, P, SZ, P]
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.hs2_block_decode_traced.argtypes = [V, P, P, I32, I32, I32, F, P, P, I32, P, P, I64, P,
                                               I32, P, P, SZ, P, I32, P]
         L.hs2_topk_select_noalloc.argtypes = [V, P, I64, I32, I32, P, I32, P, P]
+        L.hs2_noalloc_read_status.argtypes = [P]
+        L.hs2_noalloc_read_status.restype = ctypes.c_int
         L.hs2_topk_select_blocks_workspace_size.argtypes = [V, I32, I32, I32, ctypes.POINTER(SZ)]
         L.hs2_topk_select_blocks.argtypes = [V, P, I64, I32, I32, I32, P, I32, P, P, SZ, P]
         L.hs2_read_device_status.argtypes = [P, P]
@@ -170,10 +172,19 @@ class KvCache:
         return ctypes.byref(self.view)
 
 
-def workspace_size(cache: KvCache, topk: int = TOPK, window: int = WINDOW) -> int:
+WS_SCORES, WS_SELECTION = 1, 2
+
+
+def workspace_size(cache: KvCache, topk: int = TOPK, window: int = WINDOW, flags: int = 0) -> int:
+    """Workspace bytes; flags WS_SCORES / WS_SELECTION reserve room for the block outputs that
+    block_decode is given as None."""
     n = ctypes.c_size_t(0)
-    _check(lib().hs2_workspace_size(cache.ref(), topk, window, ctypes.byref(n)))
+    _check(lib().hs2_workspace_size(cache.ref(), topk, window, flags, ctypes.byref(n)))
     return int(n.value)
+
+
+def _stride0(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.stride(0)
 
 
 def _out_dtype(t: torch.Tensor) -> int:
@@ -208,6 +219,12 @@ def topk_select_noalloc(cache: KvCache, scores, idx, count, topk=TOPK, window=WI
                                          _stream(stream)))
 
 
+def noalloc_read_status(stream=None):
+    """Synchronises and raises HS2Error if the last topk_select_noalloc recorded a problem in
+    the built-in scratch (hs2_noalloc_read_status; the word is cleared by the read)."""
+    _check(lib().hs2_noalloc_read_status(_stream(stream)))
+
+
 def topk_select_blocks_workspace_size(cache: KvCache, block_size: int = 64, topk: int = TOPK,
                                       window: int = WINDOW) -> int:
     n = ctypes.c_size_t(0)
@@ -239,6 +256,8 @@ def sparse_gather_attn(cache: KvCache, q, idx, count, out, workspace, scale=None
 def block_decode(cache: KvCache, q_full, q_sparse: Sequence[torch.Tensor], out_full,
                  out_sparse: Sequence[torch.Tensor], lse, scores, idx, count, workspace,
                  topk=TOPK, window=WINDOW, scale=None, stream=None):
+    """The hybrid block (hs2_block_decode). lse, scores and idx + count may be None: the library
+    keeps them in the workspace, sized by workspace_size(..., flags=WS_SCORES | WS_SELECTION)."""
     scale = default_scale() if scale is None else scale
     L = len(q_sparse)
     if len(out_sparse) != L:
@@ -247,7 +266,7 @@ def block_decode(cache: KvCache, q_full, q_sparse: Sequence[torch.Tensor], out_f
     os_ = (ctypes.c_void_p * max(L, 1))(*[t.data_ptr() for t in out_sparse])
     _check(lib().hs2_block_decode(cache.ref(), _ptr(q_full), qs, L, topk, window, scale,
                                   _ptr(out_full), os_, _out_dtype(out_full), _ptr(lse),
-                                  _ptr(scores), scores.stride(0), _ptr(idx), idx.stride(0),
+                                  _ptr(scores), _stride0(scores), _ptr(idx), _stride0(idx),
                                   _ptr(count), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(),
                                   _stream(stream)))
@@ -267,8 +286,8 @@ def block_decode_traced(cache: KvCache, q_full, q_sparse: Sequence[torch.Tensor]
     ev = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     _check(lib().hs2_block_decode_traced(cache.ref(), _ptr(q_full), qs, L, topk, window, scale,
                                          _ptr(out_full), os_, _out_dtype(out_full), _ptr(lse),
-                                         _ptr(scores), scores.stride(0), _ptr(idx),
-                                         idx.stride(0), _ptr(count), _ptr(workspace),
+                                         _ptr(scores), _stride0(scores), _ptr(idx),
+                                         _stride0(idx), _ptr(count), _ptr(workspace),
                                          workspace.numel() * workspace.element_size(), ev,
                                          len(events), _stream(stream)))
 

@@ -647,6 +647,42 @@ BlockPlan block_plan(const Plan &P, int block_size) {
   return B;
 }
 
+// hs2_block_decode's own outputs that the caller may leave to the library: they follow the
+// workspace regions of the plan (lse always; scores and the selection when asked for).
+struct BlockExtra {
+  size_t off_lse = 0, off_scores = 0, off_idx = 0, off_count = 0, total = 0;
+  int64_t score_stride = 0;
+  int32_t idx_stride = 0;
+};
+
+constexpr uint32_t kWsFlags = HS2_WS_SCORES | HS2_WS_SELECTION;
+
+BlockExtra block_extra(const Plan &P, int topk, int window, uint32_t flags) {
+  BlockExtra E;
+  size_t o = P.total;
+  E.off_lse = o; o = align_up(o + 4 * (size_t)P.n_rows * P.H);
+  E.score_stride = (P.max_p + 1 + 63) / 64 * 64;
+  E.idx_stride = (int32_t)std::min<int64_t>(P.max_p + 1, (int64_t)topk + window);
+  E.off_scores = o;
+  if (flags & HS2_WS_SCORES) o = align_up(o + 4 * (size_t)P.n_rows * (size_t)E.score_stride);
+  E.off_idx = o;
+  if (flags & HS2_WS_SELECTION) o = align_up(o + 4 * (size_t)P.n_rows * (size_t)E.idx_stride);
+  E.off_count = o;
+  if (flags & HS2_WS_SELECTION) o = align_up(o + 4 * (size_t)P.n_rows);
+  E.total = o;
+  return E;
+}
+
+hs2_status check_ws_bytes(void *ws, size_t bytes, size_t need, uint32_t flags) {
+  if (!ws) return fail(HS2_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign)
+    return fail(HS2_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (bytes < need)
+    return fail(HS2_ERR_WORKSPACE, "workspace %zu bytes < %zu required (hs2_workspace_size with flags %u)",
+                bytes, need, flags);
+  return HS2_OK;
+}
+
 }  // namespace
 }  // namespace hs2
 
@@ -654,14 +690,16 @@ using namespace hs2;
 
 extern "C" {
 
-hs2_status hs2_workspace_size(const hs2_kv_view *kv, int32_t topk, int32_t window, size_t *bytes) {
+hs2_status hs2_workspace_size(const hs2_kv_view *kv, int32_t topk, int32_t window,
+                              uint32_t flags, size_t *bytes) {
   hs2_status st = validate_view(kv);
   if (st != HS2_OK) return st;
   if ((st = check_budget(topk, window)) != HS2_OK) return st;
   if (!bytes) return fail(HS2_ERR_INVALID_ARG, "bytes is NULL");
+  if (flags & ~kWsFlags) return fail(HS2_ERR_INVALID_ARG, "flags 0x%x: unknown bits", flags);
   Plan P;
   make_plan(kv, P);
-  *bytes = P.total;
+  *bytes = block_extra(P, topk, window, flags).total;
   return ok();
 }
 
@@ -739,6 +777,23 @@ hs2_status hs2_topk_select_noalloc(const hs2_kv_view *kv, const float *scores,
   sc.seg_info = ws_at<int2>(base, lay.off_seg_info);
   st = run_topk(kv, P, scores, score_stride, topk, window, idx, idx_stride, count, false, sc, s);
   return st == HS2_OK ? ok() : st;
+}
+
+hs2_status hs2_noalloc_read_status(void *stream) {
+  void *base = nullptr;
+  hs2_status st = noalloc_scratch(&base);
+  if (st != HS2_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_check(cudaStreamSynchronize(s), "stream synchronize")) != HS2_OK) return st;
+  uint32_t v = 0;
+  // the status word sits at the start of the built-in array (noalloc_layout's off_status)
+  if ((st = cuda_check(cudaMemcpy(&v, base, 4, cudaMemcpyDeviceToHost), "status read")) != HS2_OK)
+    return st;
+  if (v && (st = cuda_check(cudaMemset(base, 0, 4), "status clear")) != HS2_OK) return st;
+  if (v & kStatusTimeout) return fail(HS2_ERR_TIMEOUT, "a kernel's bounded wait ran out");
+  if (v & kStatusCheck)
+    return fail(HS2_ERR_DEVICE_CHECK, "a candidate score was negative or NaN");
+  return ok();
 }
 
 hs2_status hs2_topk_select_blocks_workspace_size(const hs2_kv_view *kv, int32_t block_size,
@@ -839,6 +894,22 @@ static hs2_status block_impl(const hs2_kv_view *kv, const void *q_full,
   if ((st = check_budget(topk, window)) != HS2_OK) return st;
   Plan P;
   make_plan(kv, P);
+  // outputs left NULL live in the workspace (sized by hs2_workspace_size with the same flags)
+  if ((idx == nullptr) != (count == nullptr))
+    return fail(HS2_ERR_INVALID_ARG, "idx and count must both be given or both be NULL");
+  const uint32_t flags = (scores ? 0u : (uint32_t)HS2_WS_SCORES) | (idx ? 0u : (uint32_t)HS2_WS_SELECTION);
+  const BlockExtra E = block_extra(P, topk, window, flags);
+  if ((st = check_ws_bytes(workspace, workspace_bytes, E.total, flags)) != HS2_OK) return st;
+  if (!lse) lse = ws_at<float>(workspace, E.off_lse);
+  if (!scores) {
+    scores = ws_at<float>(workspace, E.off_scores);
+    score_stride = E.score_stride;
+  }
+  if (!idx) {
+    idx = ws_at<int32_t>(workspace, E.off_idx);
+    count = ws_at<int32_t>(workspace, E.off_count);
+    idx_stride = E.idx_stride;
+  }
   if ((st = check_full_args(P, q_full, softmax_scale, out_full, out_dtype, lse, scores, score_stride)) != HS2_OK)
     return st;
   if ((st = check_idx(P, topk, window, idx, idx_stride, count)) != HS2_OK) return st;
@@ -856,7 +927,6 @@ static hs2_status block_impl(const hs2_kv_view *kv, const void *q_full,
     for (int e = 0; e < n_events; ++e)
       if (!events[e]) return fail(HS2_ERR_INVALID_ARG, "event %d is NULL", e);
   }
-  if ((st = check_ws(P, workspace, workspace_bytes)) != HS2_OK) return st;
   TensorMaps tm;
   if ((st = encode_maps(kv, tm)) != HS2_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -926,7 +996,10 @@ hs2_status hs2_read_device_status(const void *workspace, void *stream) {
   st = cuda_check(cudaMemcpy(&v, workspace, 4, cudaMemcpyDeviceToHost), "status read");
   if (st != HS2_OK) return st;
   if (v & kStatusTimeout) return fail(HS2_ERR_TIMEOUT, "a kernel's bounded wait ran out");
-  if (v & kStatusCheck) return fail(HS2_ERR_DEVICE_CHECK, "a kernel found an out-of-range index or count");
+  if (v & kStatusCheck)
+    return fail(HS2_ERR_DEVICE_CHECK,
+                "a kernel's input check failed (an out-of-range index or count, or a negative or "
+                "NaN candidate score)");
   return ok();
 }
 

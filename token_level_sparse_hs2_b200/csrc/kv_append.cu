@@ -9,9 +9,9 @@
 //
 // Each warp takes 16 (row, matrix) items, one per quarter warp per step, every load issued
 // before any store: 128 bf16 values per row, 32 per lane. bf16 cache: a copy. e4m3 cache: the row's
-// largest magnitude (half-warp max), scale = amax / 448 in float32 (1 for a zero row), codes =
-// cvt.rn.satfinite of the float32 product x * (1 / scale), the reciprocal correctly rounded
-// (round to nearest even, saturating at 448).
+// largest magnitude (quarter-warp max), scale = amax / 448 in float32 (1 for a zero row), codes =
+// cvt.rn.satfinite of the correctly rounded float32 quotient x / scale (round to nearest even,
+// saturating at 448).
 #include "common.cuh"
 #include "internal.h"
 #include "quant.cuh"
@@ -25,8 +25,8 @@ constexpr int kItemsPerStep = 32 / kLanesPerRow;       // (matrix, row) items pe
 constexpr int kSteps = 2;                              // steps per warp, loads of both first
 
 // Quarter warp q of a warp handles one (matrix, row) item per step; lane l of the quarter holds
-// values [32 l, 32 l + 32) of the row. Every per-row scalar (the destination row, the scale and
-// its reciprocal) is computed once per 8 rows of the warp, and the row maximum takes two
+// values [32 l, 32 l + 32) of the row. Every per-row scalar (the destination row and the scale)
+// is computed once per 8 rows of the warp, and the row maximum takes two
 // shuffles.
 __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ AppendParams P) {
   griddep_launch_dependents();
@@ -82,7 +82,6 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
 #pragma unroll
     for (int o = 1; o < kLanesPerRow; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sc = fp8_row_scale(amax);
-    const float inv = __frcp_rn(sc);
     uint4 c[2];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {   // 8 values -> 8 codes (2 words)
@@ -92,7 +91,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
       for (int h = 0; h < 2; ++h) {
         const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[2 * h]));
         const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[2 * h + 1]));
-        cw[h] = (fp8_pair(f0.x, f0.y, inv) & 0xffffu) | (fp8_pair(f1.x, f1.y, inv) << 16);
+        cw[h] = (fp8_pair(f0.x, f0.y, sc) & 0xffffu) | (fp8_pair(f1.x, f1.y, sc) << 16);
       }
       if (k & 1) { c[k >> 1].z = cw[0]; c[k >> 1].w = cw[1]; }
       else { c[k >> 1].x = cw[0]; c[k >> 1].y = cw[1]; }

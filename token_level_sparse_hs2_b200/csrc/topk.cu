@@ -8,7 +8,8 @@
 // (ties: lower index) are kept, then W, in ascending order.
 //
 // Scores are non-negative fp32, so their bit patterns order like their values and the
-// selection is an exact radix select on 32-bit keys:
+// selection is an exact radix select on 32-bit keys (a negative or NaN candidate score breaks
+// that order: it is recorded in the status word as a device check):
 //  1. top digit (bits 31..21) histogram: from the score pass (decode) or built here;
 //  2. the bucket B1 holding the topk-th largest key; every candidate with digit >= B1 is
 //     compacted (key, index) in position order (a ballot per warp and step and one block-wide
@@ -345,11 +346,15 @@ __global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(
   constexpr int kRegKeys = 32;
   const bool in_regs = kRegs && gh && P.seg_len <= kRegKeys * kThreadsTk;
   uint32_t rk[kRegKeys];
+  // largest key this thread reads: the bit patterns order like the values only for scores that
+  // are not negative and not NaN (keys <= 0x7f800000, +inf); anything else is reported
+  uint32_t kmax = 0;
   if (in_regs) {
 #pragma unroll
     for (int u = 0; u < kRegKeys; ++u) {
       const int64_t t = s0 + u * kThreadsTk + threadIdx.x;
       rk[u] = t < s1 ? load_key(s, t) : 0u;
+      kmax = max(kmax, rk[u]);
     }
   }
   if (gh) {
@@ -416,6 +421,7 @@ __global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(
       for (int u = 0; u < kUnroll; ++u) {
         const int64_t t = base + u * 32 + lane;
         k[u] = t < w1 ? load_key(s, t) : 0u;
+        kmax = max(kmax, k[u]);
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
@@ -469,6 +475,7 @@ __global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(
     }
     __syncthreads();
   }
+  if (kmax > 0x7f800000u) record_status(P.status, kStatusCheck);
   int n;
   if (P.n_seg == 1) {
     n = n_local;
