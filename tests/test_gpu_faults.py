@@ -63,15 +63,14 @@ def test_negative_or_nan_scores_are_reported_by_the_selection():
     """hs2_topk_select on caller scores that break the non-negative order: the call completes
     and the device status reports a check, for a split row and for many unsplit rows."""
     dev = torch.device("cuda")
-    for lens, bad in (((50000,), float("nan")), ((3000,) * 150, -0.0)):
-        w = W.make_workload(dict(name="negscore", batch=len(lens), n_q=1, n_heads=16, n_sparse=0,
-                                 kv_dtype="bf16", lengths=lens, needles=0), seed=9)
-        d = W.to_device(w, dev)
-        cache = hs2.KvCache(d["k"], d["v"], w.kv_start, w.kv_len, 1, w.n_heads)
-        s = torch.rand((len(lens), max(lens)), device=dev)
+    for lens, n_q, bad in (((50000,), 1, float("nan")), ((3000, 3100), 80, -0.0)):
+        k = torch.zeros((max(lens), 128), dtype=torch.bfloat16, device=dev)
+        cache = hs2.KvCache(k, k, [0] * len(lens), lens, n_q, 16)
+        rows = len(lens) * n_q      # 160 rows: one CTA per row; one row: split over segments
+        s = torch.rand((rows, max(lens)), device=dev)
         s[-1, 1000] = bad
-        idx = torch.empty((len(lens), 1152), dtype=torch.int32, device=dev)
-        cnt = torch.empty(len(lens), dtype=torch.int32, device=dev)
+        idx = torch.empty((rows, 1152), dtype=torch.int32, device=dev)
+        cnt = torch.empty(rows, dtype=torch.int32, device=dev)
         ws = torch.empty(hs2.workspace_size(cache), dtype=torch.uint8, device=dev)
         hs2.topk_select(cache, s, idx, cnt, ws)
         with pytest.raises(hs2.HS2Error) as e:

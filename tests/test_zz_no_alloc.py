@@ -33,20 +33,20 @@ def scores_for(lens, seed, quant):
     return s
 
 
-def cache_for(lens):
+def cache_for(lens, n_q=1):
     # the selection reads only the scores and the sequence geometry: every sequence views the
     # same rows of one small cache (rows [0, T_b)), which the view allows
     dev = torch.device("cuda")
     k = torch.zeros((max(lens), 128), dtype=torch.bfloat16, device=dev)
-    return hs2.KvCache(k, k, [0] * len(lens), lens, 1, 32), dev
+    return hs2.KvCache(k, k, [0] * len(lens), lens, n_q, 32), dev
 
 
-def compare_twice(lens, draws):
-    cache, dev = cache_for(lens)
-    B = len(lens)
+def compare_twice(lens, draws, n_q=1):
+    cache, dev = cache_for(lens, n_q)
+    B = len(lens) * n_q
     ws = torch.empty(hs2.workspace_size(cache), dtype=torch.uint8, device=dev)
     for call, (seed, quant) in enumerate(draws):
-        s = torch.from_numpy(scores_for(lens, seed, quant)).to(dev)
+        s = torch.from_numpy(scores_for(lens * n_q, seed, quant)).to(dev)
         idx_a = torch.full((B, 1152), -1, dtype=torch.int32, device=dev)
         cnt_a = torch.zeros(B, dtype=torch.int32, device=dev)
         idx_b = torch.full((B, 1152), -2, dtype=torch.int32, device=dev)
@@ -75,10 +75,8 @@ def test_noalloc_selection_over_many_segments():
 
 
 def test_noalloc_selection_many_rows():
-    # 160 rows: one CTA per row, no split
-    rng = np.random.default_rng(5)
-    lens = tuple(int(x) for x in rng.integers(900, 5000, size=160))
-    compare_twice(lens, [(31, 0), (32, 16)])
+    # 4 sequences x 40 query rows = 160 rows: one CTA per row, no split
+    compare_twice((1900, 4999, 3001, 2222), [(31, 0), (32, 16)], n_q=40)
 
 
 def test_noalloc_rejects_a_plan_above_the_builtin_scratch():

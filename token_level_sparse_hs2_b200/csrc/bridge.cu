@@ -92,6 +92,7 @@ __device__ __forceinline__ void store_row(uint32_t col, bool fp8, bool valid, ui
     return;
   }
   const float sc = fp8_row_scale(amax);
+  const float rc = fp8_row_recip(sc);
   uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {                      // 16 codes per store
@@ -100,7 +101,7 @@ __device__ __forceinline__ void store_row(uint32_t col, bool fp8, bool valid, ui
     for (int q = 0; q < 4; ++q) {
       const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&packed[8 * j + 2 * q]));
       const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&packed[8 * j + 2 * q + 1]));
-      w[q] = (fp8_pair(f0.x, f0.y, sc) & 0xffffu) | (fp8_pair(f1.x, f1.y, sc) << 16);
+      w[q] = (fp8_pair(f0.x, f0.y, sc, rc) & 0xffffu) | (fp8_pair(f1.x, f1.y, sc, rc) << 16);
     }
     d4[j] = make_uint4(w[0], w[1], w[2], w[3]);
   }

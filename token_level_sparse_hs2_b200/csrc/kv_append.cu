@@ -10,8 +10,9 @@
 // Each warp takes 16 (row, matrix) items, one per quarter warp per step, every load issued
 // before any store: 128 bf16 values per row, 32 per lane. bf16 cache: a copy. e4m3 cache: the row's
 // largest magnitude (quarter-warp max), scale = amax / 448 in float32 (1 for a zero row), codes =
-// cvt.rn.satfinite of the correctly rounded float32 quotient x / scale (round to nearest even,
-// saturating at 448).
+// cvt.rn.satfinite of the float32 quotient x / scale (round to nearest even, saturating at 448),
+// formed as in quant.cuh (a reciprocal per row, then Markstein's correction: one multiply and
+// two fused multiply-adds per value).
 #include "common.cuh"
 #include "internal.h"
 #include "quant.cuh"
@@ -82,6 +83,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
 #pragma unroll
     for (int o = 1; o < kLanesPerRow; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sc = fp8_row_scale(amax);
+    const float rc = fp8_row_recip(sc);
     uint4 c[2];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {   // 8 values -> 8 codes (2 words)
@@ -91,7 +93,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
       for (int h = 0; h < 2; ++h) {
         const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[2 * h]));
         const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[2 * h + 1]));
-        cw[h] = (fp8_pair(f0.x, f0.y, sc) & 0xffffu) | (fp8_pair(f1.x, f1.y, sc) << 16);
+        cw[h] = (fp8_pair(f0.x, f0.y, sc, rc) & 0xffffu) | (fp8_pair(f1.x, f1.y, sc, rc) << 16);
       }
       if (k & 1) { c[k >> 1].z = cw[0]; c[k >> 1].w = cw[1]; }
       else { c[k >> 1].x = cw[0]; c[k >> 1].y = cw[1]; }
