@@ -348,6 +348,14 @@ hs2_status hs2_kv_bridge(const hs2_kv_view *kv, const void *hidden, int32_t d_mo
 hs2_status hs2_selftest_wait_timeout(uint32_t limit_us, void *workspace, size_t workspace_bytes,
                                      void *stream);
 
+/* Evaluates, for the n device floats x (n >= 0), y[i] = the 2^x[i] that the tensor-core score
+ * passes compute on the FMA pipe for part of their exponentials: x clamped at -125, split as
+ * j + f with j = rint(x) and |f| <= 1/2, 2^f from a cubic fitted for minimal relative error on
+ * [-1/2, 1/2] (Remez), 2^j added to the exponent. Relative error at most 7.5e-5 for
+ * x in [-125, 0]. Not part of the method: a check of that approximation. Asynchronous on
+ * `stream`; HS2_ERR_INVALID_ARG on NULL pointers or n out of range (nothing launched). */
+hs2_status hs2_selftest_exp2(const float *x, float *y, int64_t n, void *stream);
+
 /* Number of kernels this library has launched in the calling process since it was loaded
  * (successful launches only; the workspace clears done with cudaMemsetAsync are not counted).
  * Not part of the method: an accounting aid for callers that count launches per call. */

@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.hs2_version.restype = I32
         L.hs2_launch_count.restype = ctypes.c_uint64
         L.hs2_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P, SZ, P]
+        L.hs2_selftest_exp2.argtypes = [P, P, I64, P]
+        L.hs2_selftest_exp2.restype = ctypes.c_int
         L.hs2_kv_append.argtypes = [V, P, P, P]
         L.hs2_kv_bridge.argtypes = [V, P, I32, P, P, SZ, P]
         L.hs2_kv_bridge.restype = ctypes.c_int
@@ -309,6 +311,13 @@ def selftest_wait_timeout(workspace, limit_us: int = 20000, stream=None):
                                           workspace.numel() * workspace.element_size(),
                                           _stream(stream)))
     return int(lib().hs2_read_device_status(_ptr(workspace), _stream(stream)))
+
+
+def selftest_exp2(x: torch.Tensor, y: torch.Tensor, stream=None):
+    """y = the FMA-pipe 2^x of the tensor-core score passes (hs2_selftest_exp2); fp32 tensors."""
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
+        raise ValueError("x and y must be float32 tensors of one size")
+    _check(lib().hs2_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
 
 
 def kv_append(cache: KvCache, new_k, new_v, stream=None):

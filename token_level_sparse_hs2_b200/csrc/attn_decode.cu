@@ -108,7 +108,13 @@ __device__ void produce_stream(const TensorMaps &tm, const DecodeParams &P, uint
   using C = StreamCfg<KV, HG, PASS>;
   const int lane = threadIdx.x & 31;
   TileWalk wk(P, PASS == 1);
-  if (PASS == 0) griddep_wait();   // pass 2 streams K, which no earlier kernel writes
+  // pass 1 is the block's first kernel: it waits for the previous kernel (which may have
+  // appended rows to the cache) and only then lets the next kernel start, so every later kernel
+  // of the block starts after that; pass 2 streams K without waiting
+  if (PASS == 0) {
+    griddep_wait();
+    griddep_launch_dependents();
+  }
   for (int it = 0; it < wk.n; ++it) {
     const int g = wk.step(P, it);
     const int s = it % C::kStages;
@@ -274,7 +280,6 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, (KV == kKvBf16
     fence_barrier_init();
   }
   __syncthreads();
-  griddep_launch_dependents();
   if (warp == C::kConsumers) {
     produce_stream<KV, HG, 0>(tm, P, sm.stages, sm.full, sm.empty, sm.abort_flag);
     return;
@@ -291,6 +296,7 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, (KV == kKvBf16
   WarpSoftmax st;
   st.init();
   griddep_wait();
+  griddep_launch_dependents();
   // the workspace's zero-initialised region (status word, histograms, selection counters):
   // every earlier kernel of the stream has finished, and the score pass and the selection
   // read it only after this kernel has

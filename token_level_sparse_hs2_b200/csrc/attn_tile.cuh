@@ -247,29 +247,11 @@ __device__ __forceinline__ void qk_tile_mt(const uint32_t (&qa)[MT][8][4], uint3
   }
 }
 
-// Packed fp32 pair arithmetic (sm_100): two fused multiply-adds / adds per instruction.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " mov.b64 rc, {%6, %7};\n fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}\n"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
-      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}\n"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
 // 2^x for x <= 0 on the FMA pipe (Cody-Waite split x = j + f, j = rint(x) by the 1.5 * 2^23
-// rounding trick, |f| <= 1/2): 2^f from a cubic fitted to minimise the relative error on
-// [-1/2, 1/2] (max 7.5e-5), then j is added to the exponent field. x is clamped at -125 so
-// the exponent cannot wrap; 2^-125 is far below any score's resolution.
+// rounding trick, |f| <= 1/2): 2^f from the cubic that minimises the relative error on
+// [-1/2, 1/2] (Remez exchange, tests/exp2_poly_fit.py; max 7.5e-5), then j is added to the
+// exponent field. x is clamped at -125 so the exponent cannot wrap; 2^-125 is far below any
+// score's resolution.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kMagic = 12582912.f;
   x.x = fmaxf(x.x, -125.f);
@@ -277,7 +259,7 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float2 t = fadd2(x, make_float2(kMagic, kMagic));
   const float2 r = fadd2(t, make_float2(-kMagic, -kMagic));
   const float2 f = ffma2(r, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2(f, make_float2(0.0551716648f, 0.0551716648f), make_float2(0.2426111251f, 0.2426111251f));
+  float2 p = ffma2(f, make_float2(0.0551716685f, 0.0551716685f), make_float2(0.2426111251f, 0.2426111251f));
   p = ffma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
   p = ffma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),

@@ -16,6 +16,7 @@
 #include <functional>
 #include <mutex>
 
+#include "attn_tile.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -434,22 +435,34 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   int sms = 0;
   hs2_status st = sm_count(&sms);
   if (st != HS2_OK) return st;
-  const int per_sm1 = P.kv_dtype == HS2_KV_BF16 ? 1 : 2;   // resident pass-1 CTAs per SM
-  const int G = std::max(1, std::min({per_sm1 * sms, P.total_tiles, kMaxStreamCtas}));
-  // partial slots: 4 per (CTA, sequence) pair; CTA i owns tiles [i*T/G, (i+1)*T/G)
-  const int T = P.total_tiles;
+  // 128-row tiles for the tensor-core passes
+  int t128 = 0;
+  for (int b = 0; b < P.B; ++b) {
+    dp.tile128_begin[b] = t128;
+    const int64_t r0 = kv->kv_start[b], r1 = r0 + kv->kv_len[b];
+    t128 += (int)((r1 + 127) / 128 - r0 / 128);
+  }
+  dp.tile128_begin[P.B] = t128;
+  dp.total_tiles128 = t128;
+  // pass 1: the e4m3 cache on tcgen05 (128-row tiles, one CTA per SM); the bf16 cache with
+  // warp-level products (64-row tiles, one CTA per SM)
+  const bool tc1 = P.kv_dtype == HS2_KV_FP8_E4M3;
+  const int T = tc1 ? t128 : P.total_tiles;
+  const int32_t *tb = tc1 ? dp.tile128_begin : P.tile_begin;
+  const int G = std::max(1, std::min({sms, T, kMaxStreamCtas}));
+  // partial slots: one per (CTA, sequence) pair; CTA i owns tiles [i*T/G, (i+1)*T/G)
   auto cta_of = [&](int g) { return (int)(((int64_t)(g + 1) * G - 1) / T); };
   int slots = 0;
   for (int b = 0; b < P.B; ++b) {
     dp.seq.item_begin[b] = slots;
-    slots += decode_slots_per_cta(P.H) * (cta_of(P.tile_begin[b + 1] - 1) - cta_of(P.tile_begin[b]) + 1);
+    slots += decode_slots_per_cta(P.H) * (cta_of(tb[b + 1] - 1) - cta_of(tb[b]) + 1);
   }
   dp.seq.item_begin[P.B] = slots;
   dp.batch = P.B;
   dp.n_heads = P.H;
   dp.total_tiles = T;
   dp.n_ctas = G;
-  dp.n_ctas2 = std::max(1, std::min({2 * sms, P.total_tiles, kMaxStreamCtas}));
+  dp.n_ctas2 = std::max(1, std::min(sms, t128));   // one score-pass CTA per SM
   dp.window = window;
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.kv_rows = kv->kv_rows;
@@ -469,10 +482,12 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
     dp.zero_n16 = (int32_t)(P.zero_end / 16);
   }
   if (!(passes & 1)) {   // score pass only, with the caller's lse
-    st = cuda_check(launch_decode_pass(1, P.kv_dtype, tm, dp, stream), "score pass 2");
+    st = cuda_check(launch_decode_score_tc(P.kv_dtype, tm, dp, stream), "score pass 2");
     return st;
   }
-  st = cuda_check(launch_decode_pass(0, P.kv_dtype, tm, dp, stream), "full-attention pass 1");
+  st = cuda_check(tc1 ? launch_decode_attn_fp8_tc(tm, dp, stream)
+                      : launch_decode_pass(0, P.kv_dtype, tm, dp, stream),
+                  "full-attention pass 1");
   if (st != HS2_OK) return st;
   if (mark && (st = (*mark)()) != HS2_OK) return st;
   {
@@ -490,7 +505,7 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   }
   if (mark && (st = (*mark)()) != HS2_OK) return st;
   if (!(passes & 2)) return HS2_OK;
-  st = cuda_check(launch_decode_pass(1, P.kv_dtype, tm, dp, stream), "score pass 2");
+  st = cuda_check(launch_decode_score_tc(P.kv_dtype, tm, dp, stream), "score pass 2");
   if (st != HS2_OK) return st;
   if (mark && (st = (*mark)()) != HS2_OK) return st;
   return HS2_OK;
@@ -1017,6 +1032,36 @@ __global__ void selftest_wait_kernel(uint32_t *status, uint64_t limit_ns) {
 }
 }  // namespace
 }  // namespace hs2
+
+namespace hs2 {
+namespace {
+// y = exp2_poly2(x), the FMA-pipe 2^x of the tensor-core score passes, element by element
+__global__ void selftest_exp2_kernel(const float *x, float *y, int64_t n) {
+  const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+  }
+}
+}  // namespace
+}  // namespace hs2
+
+hs2_status hs2_selftest_exp2(const float *x, float *y, int64_t n, void *stream) {
+  if (!x || !y) return fail(HS2_ERR_INVALID_ARG, "x / y is NULL");
+  if (n < 0 || n > ((int64_t)1 << 40)) return fail(HS2_ERR_INVALID_ARG, "n %lld out of range", (long long)n);
+  if (n == 0) return ok();
+  const int64_t pairs = (n + 1) / 2;
+  const int64_t blocks = (pairs + 255) / 256;
+  if (blocks > INT32_MAX) return fail(HS2_ERR_INVALID_ARG, "n too large");
+  hs2::selftest_exp2_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  hs2_status st = cuda_check(cudaGetLastError(), "exp2 self-test launch");
+  if (st != HS2_OK) return st;
+  hs2::note_launch();
+  return ok();
+}
 
 hs2_status hs2_kv_append(const hs2_kv_view *kv, const void *new_k, const void *new_v, void *stream) {
   hs2_status st = validate_view(kv);

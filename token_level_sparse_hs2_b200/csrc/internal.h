@@ -61,6 +61,10 @@ struct DecodeParams {
   uint32_t *status;
   uint4 *zero;              // pass 1: clears zero_n16 16-byte words here (the workspace's
   int32_t zero_n16;         // zero-initialised region) once the previous kernel has finished
+  // tensor-core decode kernels: 128-row tiles of all sequences, concatenated like the 64-row
+  // ones (sequence b's tiles are [tile128_begin[b], tile128_begin[b + 1]))
+  int32_t tile128_begin[HS2_MAX_BATCH + 1];
+  int32_t total_tiles128;
 };
 
 // Chunk / prefill (n_q > 1). Pass 1: blocks of 128 (query, head) rows (128 / H queries);
@@ -229,6 +233,13 @@ struct TensorMaps {
 // launchers (return cudaGetLastError() of the launch)
 cudaError_t launch_decode_pass(int pass, int kv_dtype, const TensorMaps &tm,
                                const DecodeParams &p, cudaStream_t s);
+// Score pass 2 at decode time on tcgen05 (128-row tiles; grid p.n_ctas2 persistent CTAs, one
+// per SM).
+cudaError_t launch_decode_score_tc(int kv_dtype, const TensorMaps &tm, const DecodeParams &p,
+                                   cudaStream_t s);
+// Output pass 1 at decode time for an e4m3 cache on tcgen05 (128-row tiles; grid p.n_ctas
+// persistent CTAs, one per SM; partial slots per (CTA, sequence) of that grid and tile list).
+cudaError_t launch_decode_attn_fp8_tc(const TensorMaps &tm, const DecodeParams &p, cudaStream_t s);
 cudaError_t launch_rows_pass(int pass, int kv_dtype, const TensorMaps &tm, const RowsParams &p,
                              cudaStream_t s);
 cudaError_t launch_sparse(int kv_dtype, const SparseParams &p, cudaStream_t s);
