@@ -343,8 +343,11 @@ hs2_status hs2_kv_bridge(const hs2_kv_view *kv, const void *hidden, int32_t d_mo
  * arrives at, gives up after limit_us microseconds (1 .. 2e6) and records HS2_ERR_TIMEOUT in the
  * status word at the start of `workspace` (device, 256-byte aligned, >= 256 bytes), which the
  * call clears first; hs2_read_device_status then reports HS2_ERR_TIMEOUT and the context stays
- * usable. Not part of the method: a failure-detection check. Returns HS2_ERR_WORKSPACE /
- * HS2_ERR_INVALID_ARG on bad arguments (nothing launched), HS2_ERR_CUDA on a launch error. */
+ * usable. With workspace NULL and workspace_bytes 0 the status word is the one inside the
+ * built-in array of hs2_topk_select_noalloc, which hs2_noalloc_read_status then reports (the
+ * same end-to-end check for callers that cannot allocate). Not part of the method: a
+ * failure-detection check. Returns HS2_ERR_WORKSPACE / HS2_ERR_INVALID_ARG on bad arguments
+ * (nothing launched), HS2_ERR_CUDA on a launch error. */
 hs2_status hs2_selftest_wait_timeout(uint32_t limit_us, void *workspace, size_t workspace_bytes,
                                      void *stream);
 

@@ -214,7 +214,7 @@ def test_selftest_rejects_bad_arguments_without_launching():
     import ctypes
     import token_level_sparse_hs2_b200 as hs2
     L = hs2.lib()
-    assert L.hs2_selftest_wait_timeout(1000, None, 0, None) == 3          # HS2_ERR_WORKSPACE
+    assert L.hs2_selftest_wait_timeout(1000, None, 64, None) == 3         # HS2_ERR_WORKSPACE
     buf = ctypes.create_string_buffer(1024)
     addr = (ctypes.addressof(buf) + 255) & ~255
     assert L.hs2_selftest_wait_timeout(0, ctypes.c_void_p(addr), 256, None) == 1   # limit 0

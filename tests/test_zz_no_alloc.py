@@ -109,3 +109,12 @@ def test_noalloc_reports_a_negative_score_and_clears_it():
     s[0, 777] = 1.0
     hs2.topk_select_noalloc(cache, s, idx, cnt)
     hs2.noalloc_read_status()   # a clean call reports nothing
+
+
+def test_noalloc_status_reports_a_bounded_wait_that_ran_out():
+    """The built-in array's status word carries a kernel's timeout to hs2_noalloc_read_status
+    (the self-test kernel's wait, which nothing satisfies, runs out after 20 ms), the read clears
+    it, and a selection afterwards runs and reports nothing."""
+    assert hs2.selftest_wait_timeout_noalloc(20000) == 6       # HS2_ERR_TIMEOUT
+    hs2.noalloc_read_status()                                  # cleared by the read
+    compare_twice((60003,), [(51, 0)])

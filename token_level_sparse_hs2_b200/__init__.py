@@ -320,6 +320,13 @@ def selftest_exp2(x: torch.Tensor, y: torch.Tensor, stream=None):
     _check(lib().hs2_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
 
 
+def selftest_wait_timeout_noalloc(limit_us: int = 20000, stream=None) -> int:
+    """hs2_selftest_wait_timeout on the no-allocation selection's built-in status word; returns
+    the status hs2_noalloc_read_status then reports (HS2_ERR_TIMEOUT = 6 expected)."""
+    _check(lib().hs2_selftest_wait_timeout(limit_us, None, 0, _stream(stream)))
+    return int(lib().hs2_noalloc_read_status(_stream(stream)))
+
+
 def kv_append(cache: KvCache, new_k, new_v, stream=None):
     """Writes the n_q new tokens of every sequence (bf16 [batch, n_q, 128] each) into the last
     n_q rows of each sequence of the cache (e4m3 caches: quantised with per-row scales)."""

@@ -114,7 +114,10 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
   volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + C::kStages);
   int32_t *s_idx = const_cast<int32_t *>(reinterpret_cast<volatile int32_t *>(abort_flag + 4));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x / P.n_tsplit, ts = blockIdx.x % P.n_tsplit;
+  // CTA (row, head group, split): the row's head groups are separate clusters of n_tsplit CTAs
+  const int rg = blockIdx.x / P.n_tsplit, ts = blockIdx.x % P.n_tsplit;
+  const int r = rg / P.head_groups;
+  const int hrow0 = r * P.n_heads + (rg % P.head_groups) * H;   // first (row, head) of this CTA
   const int b = r / P.n_q, i = r % P.n_q;
   const int64_t seq_row0 = P.seq.start[b];
   const int64_t p = (int64_t)P.seq.len[b] - P.n_q + i;
@@ -169,7 +172,7 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
   const int hg = warp % HG, tg = warp / HG;
   const int tok0 = tg * 16;
   const int c = lane & 3, g = lane >> 2;
-  const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(P.q) + (size_t)r * H * kHeadDim;
+  const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(P.q) + (size_t)hrow0 * kHeadDim;
   uint32_t qa[8][4];
   float rowf[2];
   if (KV == kKvBf16) {
@@ -295,8 +298,8 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
       const float Lh = hml[2 * h + 1];
       const float inv = Lh > 0.f ? 1.f / Lh : 0.f;   // 0: a shard that holds none of the selection
       if (P.lse_out && d4 == 0)
-        P.lse_out[(size_t)r * H + h] = Lh > 0.f ? (hml[2 * h] + __log2f(Lh)) * kLn2 : -INFINITY;
-      const size_t oi = ((size_t)r * H + h) * kHeadDim + 4 * d4;
+        P.lse_out[(size_t)hrow0 + h] = Lh > 0.f ? (hml[2 * h] + __log2f(Lh)) * kLn2 : -INFINITY;
+      const size_t oi = ((size_t)hrow0 + h) * kHeadDim + 4 * d4;
       if (P.out_f32) {
         *reinterpret_cast<float4 *>(reinterpret_cast<float *>(P.out) + oi) =
             make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
@@ -343,8 +346,8 @@ __global__ void __launch_bounds__(SpCfg<KV, HG>::kThreads, 2) sparse_gather_kern
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     if (P.lse_out && lane == 0)
-      P.lse_out[(size_t)r * H + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
-    const size_t oi = ((size_t)r * H + h) * kHeadDim + 4 * lane;
+      P.lse_out[(size_t)hrow0 + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+    const size_t oi = ((size_t)hrow0 + h) * kHeadDim + 4 * lane;
     if (P.out_f32) {
       *reinterpret_cast<float4 *>(reinterpret_cast<float *>(P.out) + oi) =
           make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
@@ -443,7 +446,7 @@ cudaError_t launch_sparse_t(const SparseParams &p, cudaStream_t s) {
   auto kern = sparse_gather_kernel<KV, HG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemSplit);
   if (e != cudaSuccess) return e;
-  const int grid = p.batch * p.n_q * p.n_tsplit;
+  const int grid = p.batch * p.n_q * p.head_groups * p.n_tsplit;
   if (p.n_tsplit == 1) {
     e = launch_pdl(kern, grid, C::kThreads, C::kSmem, s, p);
   } else {
@@ -507,7 +510,7 @@ int sparse_max_cluster(int kv_dtype, int n_heads) {
 }
 
 cudaError_t launch_sparse(int kv_dtype, const SparseParams &p, cudaStream_t s) {
-  const int hg = p.n_heads / 16;
+  const int hg = p.n_heads / 16 / p.head_groups;   // 16-head groups per CTA
   if (kv_dtype == HS2_KV_BF16) {
     if (hg == 1) return launch_sparse_t<kKvBf16, 1>(p, s);
     if (hg == 2) return launch_sparse_t<kKvBf16, 2>(p, s);

@@ -251,6 +251,17 @@ hs2_status encode_maps(const hs2_kv_view *kv, TensorMaps &tm) {
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
       if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled(K/V e4m3) = %d", (int)r);
     }
+    // the per-row scales, 128 rows per box (rows past kv_rows read as zero)
+    const cuuint64_t sdims[1] = {(cuuint64_t)kv->kv_rows};
+    const cuuint64_t sstrides[1] = {4};
+    const cuuint32_t sbox[1] = {128};
+    for (int which = 0; which < 2; ++which) {
+      r = g_encode(which ? &tm.vs : &tm.ks, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1,
+                   const_cast<float *>(which ? kv->v_scale : kv->k_scale), sdims, sstrides, sbox,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return fail(HS2_ERR_CUDA, "cuTensorMapEncodeTiled(scales) = %d", (int)r);
+    }
   }
   return HS2_OK;
 }
@@ -444,12 +455,13 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   }
   dp.tile128_begin[P.B] = t128;
   dp.total_tiles128 = t128;
-  // pass 1: the e4m3 cache on tcgen05 (128-row tiles, one CTA per SM); the bf16 cache with
-  // warp-level products (64-row tiles, one CTA per SM)
-  const bool tc1 = P.kv_dtype == HS2_KV_FP8_E4M3;
-  const int T = tc1 ? t128 : P.total_tiles;
-  const int32_t *tb = tc1 ? dp.tile128_begin : P.tile_begin;
-  const int G = std::max(1, std::min({sms, T, kMaxStreamCtas}));
+  // pass 1: warp-level products over 64-row tiles (one CTA per SM for bf16, two for e4m3);
+  // the score pass: the same for bf16, tcgen05 over 128-row tiles for e4m3 (one CTA per SM)
+  const bool tc2 = P.kv_dtype == HS2_KV_FP8_E4M3;
+  const int per_sm1 = P.kv_dtype == HS2_KV_BF16 ? 1 : 2;
+  const int T = P.total_tiles;
+  const int32_t *tb = P.tile_begin;
+  const int G = std::max(1, std::min({per_sm1 * sms, T, kMaxStreamCtas}));
   // partial slots: one per (CTA, sequence) pair; CTA i owns tiles [i*T/G, (i+1)*T/G)
   auto cta_of = [&](int g) { return (int)(((int64_t)(g + 1) * G - 1) / T); };
   int slots = 0;
@@ -462,7 +474,8 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   dp.n_heads = P.H;
   dp.total_tiles = T;
   dp.n_ctas = G;
-  dp.n_ctas2 = std::max(1, std::min(sms, t128));   // one score-pass CTA per SM
+  dp.n_ctas2 = tc2 ? std::max(1, std::min(sms, t128))
+                  : std::max(1, std::min({2 * sms, P.total_tiles, kMaxStreamCtas}));
   dp.window = window;
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.kv_rows = kv->kv_rows;
@@ -482,12 +495,12 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
     dp.zero_n16 = (int32_t)(P.zero_end / 16);
   }
   if (!(passes & 1)) {   // score pass only, with the caller's lse
-    st = cuda_check(launch_decode_score_tc(P.kv_dtype, tm, dp, stream), "score pass 2");
+    st = cuda_check(tc2 ? launch_decode_score_tc(P.kv_dtype, tm, dp, stream)
+                        : launch_decode_pass(1, P.kv_dtype, tm, dp, stream),
+                    "score pass 2");
     return st;
   }
-  st = cuda_check(tc1 ? launch_decode_attn_fp8_tc(tm, dp, stream)
-                      : launch_decode_pass(0, P.kv_dtype, tm, dp, stream),
-                  "full-attention pass 1");
+  st = cuda_check(launch_decode_pass(0, P.kv_dtype, tm, dp, stream), "full-attention pass 1");
   if (st != HS2_OK) return st;
   if (mark && (st = (*mark)()) != HS2_OK) return st;
   {
@@ -505,7 +518,9 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   }
   if (mark && (st = (*mark)()) != HS2_OK) return st;
   if (!(passes & 2)) return HS2_OK;
-  st = cuda_check(launch_decode_score_tc(P.kv_dtype, tm, dp, stream), "score pass 2");
+  st = cuda_check(tc2 ? launch_decode_score_tc(P.kv_dtype, tm, dp, stream)
+                      : launch_decode_pass(1, P.kv_dtype, tm, dp, stream),
+                  "score pass 2");
   if (st != HS2_OK) return st;
   if (mark && (st = (*mark)()) != HS2_OK) return st;
   return HS2_OK;
@@ -576,11 +591,16 @@ hs2_status run_sparse(const hs2_kv_view *kv, const Plan &P, const void *q, const
   const int64_t cap = std::min<int64_t>(idx_stride, P.max_p + 1);
   const int tiles = (int)((cap + kTile - 1) / kTile);
   int ts = 1;
+  sp.head_groups = 1;
   if (P.sparse_split) {   // about one CTA per SM: spread the gather over the chip
+    // few rows: the heads too are split, two 16-head CTAs (separate clusters) per row, each
+    // gathering the row's selection for its heads (the second read of a row hits L2)
+    sp.head_groups = P.H / 16;
+    const int units = P.n_rows * sp.head_groups;
     int max_cluster = 1;
-    hs2_status st = sparse_cluster_limit(P.kv_dtype, P.H, &max_cluster);
+    hs2_status st = sparse_cluster_limit(P.kv_dtype, P.H / sp.head_groups, &max_cluster);
     if (st != HS2_OK) return st;
-    ts = std::max(1, std::min({(kManyRows + P.n_rows - 1) / P.n_rows, tiles, kMaxSplit, max_cluster}));
+    ts = std::max(1, std::min({(kManyRows + units - 1) / units, tiles, kMaxSplit, max_cluster}));
   }
   const int tiles_per = (tiles + ts - 1) / ts;
   sp.split_len = tiles_per * kTile;
@@ -1320,9 +1340,14 @@ hs2_status hs2_kv_bridge(const hs2_kv_view *kv, const void *hidden, int32_t d_mo
 
 hs2_status hs2_selftest_wait_timeout(uint32_t limit_us, void *workspace, size_t workspace_bytes,
                                      void *stream) {
+  if (limit_us < 1 || limit_us > 2000000) return fail(HS2_ERR_INVALID_ARG, "limit_us %u outside [1, 2e6]", limit_us);
+  if (!workspace && workspace_bytes == 0) {   // the no-allocation selection's built-in status word
+    hs2_status st = noalloc_scratch(&workspace);
+    if (st != HS2_OK) return st;
+    workspace_bytes = HS2_NOALLOC_SCRATCH_BYTES;
+  }
   if (!workspace || workspace_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return fail(HS2_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold 256 bytes");
-  if (limit_us < 1 || limit_us > 2000000) return fail(HS2_ERR_INVALID_ARG, "limit_us %u outside [1, 2e6]", limit_us);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   hs2_status st = cuda_check(cudaMemsetAsync(workspace, 0, 4, s), "status clear");
   if (st != HS2_OK) return st;

@@ -90,11 +90,12 @@ struct RowsParams {
   uint32_t *status;
 };
 
-// Sparse gather attention: one CTA per (query row, split of the selected list).
+// Sparse gather attention: one CTA per (query row, head group, split of the selected list).
 struct SparseParams {
   SeqTable seq;
   int32_t batch, n_q, n_heads;
   int32_t n_tsplit;         // CTAs per row along the selected list (one thread-block cluster)
+  int32_t head_groups;      // CTAs (clusters) per row across the heads: 1, or 2 of 16 heads
   int32_t split_len;        // selected entries per CTA (multiple of 64)
   float scale_log2;
   const void *q;            // bf16 [B, n_q, H, 128]
@@ -228,18 +229,16 @@ cudaError_t launch_cp_localize(const CpParams &p, cudaStream_t s);
 
 struct TensorMaps {
   CUtensorMap k, v;
+  CUtensorMap ks, vs;         // e4m3 caches: the per-row scales as 1-D tensors (boxes of 128)
 };
 
 // launchers (return cudaGetLastError() of the launch)
 cudaError_t launch_decode_pass(int pass, int kv_dtype, const TensorMaps &tm,
                                const DecodeParams &p, cudaStream_t s);
-// Score pass 2 at decode time on tcgen05 (128-row tiles; grid p.n_ctas2 persistent CTAs, one
-// per SM).
+// Score pass 2 at decode time for an e4m3 cache on tcgen05 (128-row tiles; grid p.n_ctas2
+// persistent CTAs, one per SM; kv_dtype must be HS2_KV_FP8_E4M3).
 cudaError_t launch_decode_score_tc(int kv_dtype, const TensorMaps &tm, const DecodeParams &p,
                                    cudaStream_t s);
-// Output pass 1 at decode time for an e4m3 cache on tcgen05 (128-row tiles; grid p.n_ctas
-// persistent CTAs, one per SM; partial slots per (CTA, sequence) of that grid and tile list).
-cudaError_t launch_decode_attn_fp8_tc(const TensorMaps &tm, const DecodeParams &p, cudaStream_t s);
 cudaError_t launch_rows_pass(int pass, int kv_dtype, const TensorMaps &tm, const RowsParams &p,
                              cudaStream_t s);
 cudaError_t launch_sparse(int kv_dtype, const SparseParams &p, cudaStream_t s);
