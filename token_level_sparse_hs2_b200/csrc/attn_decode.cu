@@ -36,20 +36,28 @@ struct StreamCfg {
   static constexpr int kPass1Rows = (KV == kKvBf16) ? 64 : 32;
   static constexpr int kPass1Warps = (KV == kKvBf16) ? 6 : 4;
   static constexpr int kPass2Rows = 32;   // tile rows per pass-2 warp (all heads)
-  static constexpr int kGroupWarps = (PASS == 0) ? (kTile / kPass1Rows) * HG : kTile / kPass2Rows;
-  static constexpr int kGroups = (PASS == 0) ? kPass1Warps / kGroupWarps : 4 / kGroupWarps;
+  // 64-row tiles per pipeline stage (kSub > 1: one CTA per SM moving kSub tiles a stage, with
+  // 4 * kSub consumer warps; measured no faster than two CTAs per SM of single-tile stages)
+#ifndef HS2_PASS2_SUB
+#define HS2_PASS2_SUB 1
+#endif
+  static constexpr int kSub = (KV == kKvBf16 && PASS == 1) ? HS2_PASS2_SUB : 1;
+  static constexpr int kPass2Warps = (kSub == 2) ? 8 : 4;
+  static constexpr int kGroupWarps = (PASS == 0) ? (kTile / kPass1Rows) * HG : kSub * (kTile / kPass2Rows);
+  static constexpr int kGroups = (PASS == 0) ? kPass1Warps / kGroupWarps : kPass2Warps / kGroupWarps;
   static constexpr int kConsumers = kGroupWarps * kGroups;
   static constexpr int kThreads = (kConsumers + 1) * 32;
   static constexpr int kKBytes = (KV == kKvBf16) ? 2 * kBoxBytes : kBoxBytes;
   static constexpr int kVBytes = (PASS == 0) ? kKBytes : 0;
   static constexpr int kScaleBytes = (KV == kKvFp8) ? (PASS == 0 ? 512 : 256) : 0;
-  static constexpr int kStageBytes = (kKBytes + kVBytes + kScaleBytes + 1023) / 1024 * 1024;
-  static constexpr int kStages = (KV == kKvBf16) ? (PASS == 0 ? 6 : 4) : (PASS == 0 ? 4 : 6);
+  static constexpr int kTileBytes = kKBytes + kVBytes + kScaleBytes;   // one 64-row tile
+  static constexpr int kStageBytes = (kSub * kTileBytes + 1023) / 1024 * 1024;
+  static constexpr int kStages = (KV == kKvBf16) ? (PASS == 0 || kSub > 1 ? 6 : 4) : (PASS == 0 ? 4 : 6);
   // Stage s is refilled for steps s, s + kStages, ...; with kStages a multiple of kGroups all
   // of those steps belong to one group, so a group never waits on a stage whose previous fill
   // another group has not consumed yet (a parity wait cannot tell fill f from fill f + 2).
   static_assert(kStages % kGroups == 0, "stages must be a multiple of the consumer groups");
-  static constexpr uint32_t kTxBytes = kKBytes + kVBytes;
+  static constexpr uint32_t kTxBytes = kKBytes + kVBytes;   // TMA bytes per 64-row tile
   static constexpr uint32_t kFullCount = (KV == kKvFp8) ? 33 : 1;
   // pass 1: the consumer warps' partials of a sequence merge in shared memory ([H][128] output
   // sums, then [8 warps][16 rows] max and denominator) before one partial per CTA is written
@@ -115,11 +123,11 @@ __device__ void produce_stream(const TensorMaps &tm, const DecodeParams &P, uint
     griddep_wait();
     griddep_launch_dependents();
   }
-  for (int it = 0; it < wk.n; ++it) {
-    const int g = wk.step(P, it);
-    const int s = it % C::kStages;
-    const uint32_t par = ((it / C::kStages) & 1) ^ 1;
-    if (it >= C::kStages) {
+  const int n_stages = (wk.n + C::kSub - 1) / C::kSub;
+  for (int k = 0; k < n_stages; ++k) {
+    const int s = k % C::kStages;
+    const uint32_t par = ((k / C::kStages) & 1) ^ 1;
+    if (k >= C::kStages) {
       bool ok = true;
       if (lane == 0) ok = mbar_wait(smem_u32(&empty[s]), par);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -132,12 +140,15 @@ __device__ void produce_stream(const TensorMaps &tm, const DecodeParams &P, uint
       }
     }
     if (*abort_flag) return;
-    uint8_t *st = stages + s * C::kStageBytes;
     const uint32_t bar = smem_u32(&full[s]);
+    const int nsub = min(C::kSub, wk.n - k * C::kSub);
+    if (lane == 0) mbar_arrive_expect_tx(bar, nsub * C::kTxBytes);
+    for (int u = 0; u < nsub; ++u) {
+    const int g = wk.step(P, k * C::kSub + u);
+    uint8_t *st = stages + s * C::kStageBytes + u * C::kTileBytes;
     const int64_t y64 = tile_row0(P, wk.b, g);
     const int y = (int)y64;
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar, C::kTxBytes);
       if (KV == kKvBf16) {
         tma_load_2d(smem_u32(st), &tm.k, bar, 0, y);
         tma_load_2d(smem_u32(st + kBoxBytes), &tm.k, bar, 64, y);
@@ -162,6 +173,7 @@ __device__ void produce_stream(const TensorMaps &tm, const DecodeParams &P, uint
           cp_async_4(smem_u32(sc + (kTile + rr) * 4), P.v_scale + (in ? row : 0), in ? 4u : 0u);
       }
       cp_async_mbar_arrive(bar);
+    }
     }
   }
 }
@@ -356,7 +368,7 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, (KV == kKvBf16
 // ------------------------------------------------------------------ pass 2
 
 template <int KV, int HG>
-__global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, 2)
+__global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, StreamCfg<KV, HG, 1>::kSub > 1 ? 1 : 2)
     decode_pass2_kernel(const __grid_constant__ TensorMaps tm, const __grid_constant__ DecodeParams P) {
   using C = StreamCfg<KV, HG, 1>;
   constexpr int H = 16 * HG;
@@ -384,17 +396,30 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, 2)
     const int grp = warp / C::kGroupWarps, gw = warp % C::kGroupWarps;
     const int g8 = lane >> 2, c = lane & 3;
     constexpr int NT2 = C::kPass2Rows / 8;
-    const int tok0 = gw * C::kPass2Rows;
+    constexpr int kWarpsPerTile = kTile / C::kPass2Rows;
+    const int sub = gw / kWarpsPerTile;                       // this warp's tile of each stage
+    const int tok0 = (gw % kWarpsPerTile) * C::kPass2Rows;    // and its rows in that tile
     int cur = -1;
     int64_t n_cand = 0;
     uint32_t *hrow = nullptr;
     uint32_t qa[HG][8][4];
     float rowf[HG][2], lse2[HG][2];
     griddep_wait();
-    for (int it = 0; it < wk.n; ++it) {
+    const int n_stages = (wk.n + C::kSub - 1) / C::kSub;
+    for (int k = grp; k < n_stages; k += C::kGroups) {
+      const int it = k * C::kSub + sub;
+      const int s = k % C::kStages;
+      if (it >= wk.n) {   // the last stage holds fewer tiles: release it all the same
+        if (!mbar_wait(smem_u32(&sm.full[s]), (k / C::kStages) & 1)) {
+          record_status(P.status, kStatusTimeout);
+          *sm.abort_flag = 1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+        continue;
+      }
       const int g = wk.step(P, it);
       const int b = wk.b;
-      if (it % C::kGroups != grp) continue;
       if (b != cur) {
         cur = b;
         const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(P.q) + (size_t)b * H * kHeadDim;
@@ -408,13 +433,12 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 1>::kThreads, 2)
         hrow = (b - b_lo < 2) ? sm.hist + (b - b_lo) * kHistBins
                               : (P.hist ? P.hist + (size_t)b * kHistBins : nullptr);
       }
-      const int s = it % C::kStages;
-      if (!mbar_wait(smem_u32(&sm.full[s]), (it / C::kStages) & 1)) {
+      if (!mbar_wait(smem_u32(&sm.full[s]), (k / C::kStages) & 1)) {
         record_status(P.status, kStatusTimeout);
         *sm.abort_flag = 1;
       }
       if (*sm.abort_flag) break;
-      const uint8_t *stg = sm.stages + s * C::kStageBytes;
+      const uint8_t *stg = sm.stages + s * C::kStageBytes + sub * C::kTileBytes;
       const int64_t trow = tile_row0(P, b, g);
       const int64_t row0 = P.seq.start[b], row1 = row0 + P.seq.len[b];
       float colk[NT2][2];

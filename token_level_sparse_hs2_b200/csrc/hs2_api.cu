@@ -474,8 +474,9 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   dp.n_heads = P.H;
   dp.total_tiles = T;
   dp.n_ctas = G;
-  dp.n_ctas2 = tc2 ? std::max(1, std::min(sms, t128))
-                  : std::max(1, std::min({2 * sms, P.total_tiles, kMaxStreamCtas}));
+  dp.n_ctas2 = tc2 ? std::max(1, std::min(sms, t128))                 // one CTA per SM
+                  : (HS2_PASS2_SUB > 1 ? std::max(1, std::min(sms, (P.total_tiles + 1) / 2))
+                                       : std::max(1, std::min({2 * sms, P.total_tiles, kMaxStreamCtas})));
   dp.window = window;
   dp.scale_log2 = scale * 1.4426950408889634f;
   dp.kv_rows = kv->kv_rows;

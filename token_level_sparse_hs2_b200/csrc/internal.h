@@ -235,6 +235,10 @@ struct TensorMaps {
 // launchers (return cudaGetLastError() of the launch)
 cudaError_t launch_decode_pass(int pass, int kv_dtype, const TensorMaps &tm,
                                const DecodeParams &p, cudaStream_t s);
+// Tiles per stage of the bf16 decode score pass (one CTA per SM when above 1, else two).
+#ifndef HS2_PASS2_SUB
+#define HS2_PASS2_SUB 1
+#endif
 // Score pass 2 at decode time for an e4m3 cache on tcgen05 (128-row tiles; grid p.n_ctas2
 // persistent CTAs, one per SM; kv_dtype must be HS2_KV_FP8_E4M3).
 cudaError_t launch_decode_score_tc(int kv_dtype, const TensorMaps &tm, const DecodeParams &p,
