@@ -19,7 +19,9 @@
 //    scaling (a bf16 value has 8 significant bits, hi takes 4 and the remainder needs at most
 //    4), so D = K.(hi + lo) equals K.Q 2^-e_h but for elements of magnitude below 2^-2
 //    (2^-9 .. 2^-8 of the head's largest), whose remainder is rounded in e4m3's subnormal
-//    range (error at most 2^-10 each). The logit is D k_scale[t] c 2^e_h.
+//    range (error at most 2^-10 each). The hi terms are the operand's rows [0, H) and the lo
+//    terms its rows [H, 2H), so one product of N = 2H reads each K tile once and the epilogue
+//    adds a head's two columns. The logit is (D_h + D_{H+h}) k_scale[t] c 2^e_h.
 //
 // Persistent grid, one CTA per SM: CTA i walks an equal contiguous range of the concatenated
 // 128-row tiles of all sequences, in reverse (pass 1 read those rows last; some are still in
@@ -46,9 +48,17 @@ constexpr int kDtGroups = 2;                    // epilogue groups, alternate ti
 constexpr int kDtEpiWarps = 4 * kDtGroups;
 constexpr int kDtWarpMma = kDtEpiWarps, kDtWarpTma = kDtEpiWarps + 1;
 constexpr int kDtThreads = (kDtEpiWarps + 2) * 32;
-constexpr int kDtAcc = 4;                       // accumulators of 32 columns
-constexpr uint32_t kDtCols = 32 * kDtAcc;
-constexpr int kDtQSlot = 32 * 256;              // a sequence's query operand (H <= 32 rows)
+constexpr int kDtAcc = 4;                       // accumulators in TMEM
+constexpr int kDtQSlot = 32 * 256;              // a sequence's query operand (2H <= 64 rows)
+
+// The product's N (bf16: the H heads; e4m3: H hi rows, then H lo rows) and the TMEM columns
+// one accumulator takes (at least 32, so that every allocation is a power of two).
+template <int KV, int H>
+struct DtCols {
+  static constexpr int kN = (KV == kKvFp8) ? 2 * H : H;
+  static constexpr uint32_t kAcc = kN < 32 ? 32 : kN;
+  static constexpr uint32_t kAll = kAcc * kDtAcc;
+};
 
 template <int KV>
 struct DtCfg {
@@ -177,7 +187,8 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint
 }
 
 // The query operand of sequence b in a slot, K-major with the 128-byte swizzle, one lane per
-// head. bf16: two [32][128 B] halves (dims 0..63, 64..127). e4m3: hi [32][128 B], then lo.
+// head. bf16: two [32][128 B] halves (dims 0..63, 64..127). e4m3: one [2H][128 B] block, hi in
+// row h and lo in row H + h.
 template <int KV, int H>
 __device__ void dt_prep_q(const DecodeParams &P, int b, uint8_t *slot) {
   const int h = threadIdx.x & 31;
@@ -189,11 +200,15 @@ __device__ void dt_prep_q(const DecodeParams &P, int b, uint8_t *slot) {
       for (int c = 0; c < 16; ++c)
         *reinterpret_cast<uint4 *>(slot + (c >> 3) * (32 * 128) + sw128(h, (c & 7) * 16)) = q[c];
     } else {
+      // one lane works through its head's 128 dims alone: all loads in flight at once and the
+      // loops unrolled, so that the chain is short
+      uint4 qv[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) qv[c] = q[c];
       float amax = 0.f;
-#pragma unroll 4
+#pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const uint4 v = q[c];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
@@ -202,11 +217,9 @@ __device__ void dt_prep_q(const DecodeParams &P, int b, uint8_t *slot) {
       }
       const int ex = amax > 0.f ? ilogbf(amax) - 7 : 0;   // largest |q 2^-ex| in [128, 256)
       const float down = ldexpf(1.f, -ex);
-      uint8_t *hi_row = slot, *lo_row = slot + 32 * 128;
-#pragma unroll 2
+#pragma unroll
       for (int c = 0; c < 16; ++c) {   // 8 dims: 8 hi codes, 8 lo codes
-        const uint4 v = q[c];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
         uint32_t hc[2], lc[2];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -227,8 +240,8 @@ __device__ void dt_prep_q(const DecodeParams &P, int b, uint8_t *slot) {
             lc[word] |= (uint32_t)lo << 16;
           }
         }
-        *reinterpret_cast<uint2 *>(hi_row + sw128(h, c * 8)) = make_uint2(hc[0], hc[1]);
-        *reinterpret_cast<uint2 *>(lo_row + sw128(h, c * 8)) = make_uint2(lc[0], lc[1]);
+        *reinterpret_cast<uint2 *>(slot + sw128(h, c * 8)) = make_uint2(hc[0], hc[1]);
+        *reinterpret_cast<uint2 *>(slot + sw128(H + h, c * 8)) = make_uint2(lc[0], lc[1]);
       }
     }
   }
@@ -247,11 +260,13 @@ __device__ void dt_seq_consts(const DecodeParams &P, int b, float *cst, float (&
     if (KV == kKvFp8) {   // the same power of two dt_prep_q takes out of the head
       const uint4 *q = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(P.q) +
                                                        ((size_t)b * H + h) * kHeadDim);
+      uint4 qv[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) qv[c] = q[c];
       float amax = 0.f;
-#pragma unroll 4
+#pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const uint4 v = q[c];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
@@ -277,6 +292,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     decode_score_tc_kernel(const __grid_constant__ TensorMaps tm, const __grid_constant__ DecodeParams P) {
   using C = DtCfg<KV>;
   constexpr int H = 16 * HG;
+  using N = DtCols<KV, H>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   DtSmem<KV> sm(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -298,7 +314,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   }
   for (int t = threadIdx.x; t < 2 * kHistBins; t += kDtThreads) sm.hist[t] = 0;
   if (warp == kDtWarpMma) {
-    tmem_alloc(smem_u32(sm.tmem_base), kDtCols);
+    tmem_alloc(smem_u32(sm.tmem_base), N::kAll);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -343,13 +359,17 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     __syncwarp();
   } else if (warp == kDtWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    griddep_wait();
-    const uint32_t idesc = (KV == kKvBf16) ? umma_idesc_bf16(kDt, H) : umma_idesc_e4m3(kDt, H);
+    // The queries are an input of the block (no kernel before this one in the block writes
+    // them, and the block's first kernel starts only after everything before the block has
+    // ended), so the first operand is laid out while the previous kernel finishes; the lse
+    // the epilogue reads is that kernel's output.
+    const uint32_t idesc = (KV == kKvBf16) ? umma_idesc_bf16(kDt, N::kN) : umma_idesc_e4m3(kDt, N::kN);
     int cur = -1, prepped = -1, last_seq_it = -1;
     if (wk.n > 0) {
       dt_prep_q<KV, H>(P, wk.b, sm.q);
       prepped = 0;
     }
+    griddep_wait();
     int b_next = -1;   // the sequence after the current one in the walk, if any
     for (int it = 0; it < wk.n; ++it) {
       const int g = wk.step(P, it);
@@ -366,7 +386,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
       if (lane == 0) {
         const uint32_t st = smem_u32(sm.stages + s * C::kStageBytes);
         const uint32_t qs = smem_u32(sm.q + (cur & 1) * kDtQSlot);
-        const uint32_t d = tmem + a * 32;
+        const uint32_t d = tmem + a * N::kAcc;
         if (KV == kKvBf16) {
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
@@ -376,11 +396,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
           }
         } else {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {   // hi terms, then lo terms
-            const uint32_t off = (k & 3) * 32;
-            const uint32_t qoff = (k >> 2) * (32 * 128) + (k & 3) * 32;
-            umma_e4m3(d, umma_desc_sw128(st + off, 1024), umma_desc_sw128(qs + qoff, 1024), idesc, k > 0);
-          }
+          for (int k = 0; k < 4; ++k)   // 32 dims a step; hi and lo terms in one product
+            umma_e4m3(d, umma_desc_sw128(st + k * 32, 1024), umma_desc_sw128(qs + k * 32, 1024), idesc, k > 0);
         }
         umma_commit(smem_u32(&sm.empty[s]));
         umma_commit(smem_u32(&sm.acc_full[a]));
@@ -429,8 +446,9 @@ __global__ void __launch_bounds__(kDtThreads, 1)
       const int s = it % C::kStages, a = it % kDtAcc;
       if (!dt_wait(P, sm.abort_flag, &sm.acc_full[a], (it / kDtAcc) & 1)) break;
       tc_fence_after();
-      float v[32];
-      tmem_ld32(lane_addr + a * 32, v);
+      float v[32], w[32];   // e4m3: v the hi columns, w the lo columns (H = 32); or v both (H = 16)
+      tmem_ld32(lane_addr + a * N::kAcc, v);
+      if (KV == kKvFp8 && H == 32) tmem_ld32(lane_addr + a * N::kAcc + 32, w);
       float ks = 1.f;
       if (KV == kKvFp8)
         ks = reinterpret_cast<const float *>(sm.stages + s * C::kStageBytes + C::kCodeBytes)[tok];
@@ -446,9 +464,13 @@ __global__ void __launch_bounds__(kDtThreads, 1)
 #pragma unroll
       for (int i = 0; i < H / 2; ++i) {
         float2 m = make_float2(a_h[2 * i], a_h[2 * i + 1]);
-        if (KV == kKvFp8) m = fmul2(m, make_float2(ks, ks));
-        const float2 x = ffma2(make_float2(v[2 * i], v[2 * i + 1]), m,
-                               make_float2(-l2_h[2 * i], -l2_h[2 * i + 1]));
+        float2 d = make_float2(v[2 * i], v[2 * i + 1]);
+        if (KV == kKvFp8) {
+          m = fmul2(m, make_float2(ks, ks));
+          d = fadd2(d, H == 32 ? make_float2(w[2 * i], w[2 * i + 1])
+                               : make_float2(v[(H + 2 * i) & 31], v[(H + 2 * i + 1) & 31]));
+        }
+        const float2 x = ffma2(d, m, make_float2(-l2_h[2 * i], -l2_h[2 * i + 1]));
         acc = fadd2(acc, make_float2(fast_exp2(x.x), fast_exp2(x.y)));
       }
       const float sc = acc.x + acc.y;
@@ -472,7 +494,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   }
   if (warp == kDtWarpMma) {
     tc_fence_after();
-    tmem_dealloc(tmem, kDtCols);
+    tmem_dealloc(tmem, N::kAll);
   }
 }
 
