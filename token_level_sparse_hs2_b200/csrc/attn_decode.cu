@@ -86,10 +86,22 @@ struct TileWalk {
   int lo, hi, n;
   bool reverse;
   int b;
-  __device__ TileWalk(const DecodeParams &P, bool rev) {
-    const int G = gridDim.x, T = P.total_tiles;
-    lo = range_lo(blockIdx.x, G, T);
-    hi = range_lo(blockIdx.x + 1, G, T);
+  __device__ TileWalk(const DecodeParams &P, bool rev, bool per_seq = false) {
+    if (per_seq) {   // the CTA's share of its own sequence's tiles
+      int s0 = 0, s1 = P.batch - 1;
+      while (s0 < s1) {
+        const int mid = (s0 + s1 + 1) >> 1;
+        if (P.cta_begin[mid] <= (int)blockIdx.x) s0 = mid; else s1 = mid - 1;
+      }
+      const int nc = P.cta_begin[s0 + 1] - P.cta_begin[s0], j = (int)blockIdx.x - P.cta_begin[s0];
+      const int t0 = P.seq.tile_begin[s0], nt = P.seq.tile_begin[s0 + 1] - t0;
+      lo = t0 + (int)((int64_t)j * nt / nc);
+      hi = t0 + (int)((int64_t)(j + 1) * nt / nc);
+    } else {
+      const int G = gridDim.x, T = P.total_tiles;
+      lo = range_lo(blockIdx.x, G, T);
+      hi = range_lo(blockIdx.x + 1, G, T);
+    }
     n = hi - lo;
     reverse = rev;
     b = (n > 0) ? seq_of_tile(P.seq, P.batch, reverse ? hi - 1 : lo) : 0;
@@ -115,7 +127,7 @@ __device__ void produce_stream(const TensorMaps &tm, const DecodeParams &P, uint
                                uint64_t *full, uint64_t *empty, volatile int *abort_flag) {
   using C = StreamCfg<KV, HG, PASS>;
   const int lane = threadIdx.x & 31;
-  TileWalk wk(P, PASS == 1);
+  TileWalk wk(P, PASS == 1, PASS == 0 && P.seq_split);
   // pass 1 is the block's first kernel: it waits for the previous kernel (which may have
   // appended rows to the cache) and only then lets the next kernel start, so every later kernel
   // of the block starts after that; pass 2 streams K without waiting
@@ -253,7 +265,7 @@ __device__ void flush_partial(const DecodeParams &P, int b, int hg, const WarpSo
     if (warp / HG == k) o_to_smem<KV>(mo + hg * 16 * o_stride<KV>(), st.o, f, k == 0);
     named_barrier_sync(1, NT);
   }
-  const int first = cta_of_tile(P.seq.tile_begin[b], gridDim.x, P.total_tiles);
+  const int first = P.seq_split ? P.cta_begin[b] : cta_of_tile(P.seq.tile_begin[b], gridDim.x, P.total_tiles);
   const int slot = P.seq.item_begin[b] + (blockIdx.x - first);
   float *part = P.part + (size_t)slot * H * kPartRow;
   for (int t = threadIdx.x; t < H * kHeadDim / 4; t += NT) {
@@ -301,7 +313,7 @@ __global__ void __launch_bounds__(StreamCfg<KV, HG, 0>::kThreads, (KV == kKvBf16
   constexpr int NT = C::kPass1Rows / 8;
   const int tok0 = tg * C::kPass1Rows;
   const int c = lane & 3;
-  TileWalk wk(P, false);
+  TileWalk wk(P, false, P.seq_split != 0);
   int cur = -1;
   uint32_t qa[8][4];
   float rowf[2];

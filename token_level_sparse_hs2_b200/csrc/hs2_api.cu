@@ -388,6 +388,44 @@ hs2_status sm_count(int *out) {
 
 // ------------------------------------------------------------------ steps
 
+// Pass 1 can give every sequence of a batch CTAs of its own: a CTA whose tiles cross a sequence
+// boundary stops all its warps for a mid-range flush of their partials and a new query, which
+// measured about the time of seven tiles, so the split is taken whenever no CTA gets more than
+// three tiles above the contiguous split's share. CTAs go to sequences by their tiles (at least
+// one each, never more than the sequence has tiles, the rest by largest remainder); the grid
+// is the number of CTAs handed out. cta_begin gets B + 1 prefix offsets.
+static bool pass1_seq_split(int B, const int32_t *tb, int G, int32_t *cta_begin) {
+  const int T = tb[B];
+  if (B < 2 || B > G || T < 1) return false;
+  int n[HS2_MAX_BATCH];
+  double rem[HS2_MAX_BATCH];
+  int used = 0;
+  for (int b = 0; b < B; ++b) {
+    const int nt = tb[b + 1] - tb[b];
+    if (nt < 1) return false;
+    const double share = (double)G * nt / T;
+    n[b] = std::min(nt, std::max(1, (int)share));
+    rem[b] = share - n[b];
+    used += n[b];
+  }
+  if (used > G) return false;
+  while (used < G) {
+    int best = -1;
+    for (int b = 0; b < B; ++b)
+      if (n[b] < tb[b + 1] - tb[b] && (best < 0 || rem[b] > rem[best])) best = b;
+    if (best < 0) break;
+    ++n[best];
+    rem[best] -= 1.0;
+    ++used;
+  }
+  int most = 0;
+  for (int b = 0; b < B; ++b) most = std::max(most, (tb[b + 1] - tb[b] + n[b] - 1) / n[b]);
+  if (most > (T + G - 1) / G + 3) return false;
+  cta_begin[0] = 0;
+  for (int b = 0; b < B; ++b) cta_begin[b + 1] = cta_begin[b] + n[b];
+  return true;
+}
+
 hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, const void *q,
                     float scale, void *out, int out_f32, float *lse, float *scores,
                     int64_t score_stride, int window, bool with_hist, void *ws,
@@ -461,15 +499,22 @@ hs2_status run_full(const hs2_kv_view *kv, const Plan &P, const TensorMaps &tm, 
   const int per_sm1 = P.kv_dtype == HS2_KV_BF16 ? 1 : 2;
   const int T = P.total_tiles;
   const int32_t *tb = P.tile_begin;
-  const int G = std::max(1, std::min({per_sm1 * sms, T, kMaxStreamCtas}));
-  // partial slots: one per (CTA, sequence) pair; CTA i owns tiles [i*T/G, (i+1)*T/G)
-  auto cta_of = [&](int g) { return (int)(((int64_t)(g + 1) * G - 1) / T); };
-  int slots = 0;
-  for (int b = 0; b < P.B; ++b) {
-    dp.seq.item_begin[b] = slots;
-    slots += decode_slots_per_cta(P.H) * (cta_of(tb[b + 1] - 1) - cta_of(tb[b]) + 1);
+  int G = std::max(1, std::min({per_sm1 * sms, T, kMaxStreamCtas}));
+  if (pass1_seq_split(P.B, tb, G, dp.cta_begin)) {
+    // every CTA in one sequence: its partial slot is its index
+    dp.seq_split = 1;
+    G = dp.cta_begin[P.B];
+    for (int b = 0; b <= P.B; ++b) dp.seq.item_begin[b] = dp.cta_begin[b];
+  } else {
+    // partial slots: one per (CTA, sequence) pair; CTA i owns tiles [i*T/G, (i+1)*T/G)
+    auto cta_of = [&](int g) { return (int)(((int64_t)(g + 1) * G - 1) / T); };
+    int slots = 0;
+    for (int b = 0; b < P.B; ++b) {
+      dp.seq.item_begin[b] = slots;
+      slots += decode_slots_per_cta(P.H) * (cta_of(tb[b + 1] - 1) - cta_of(tb[b]) + 1);
+    }
+    dp.seq.item_begin[P.B] = slots;
   }
-  dp.seq.item_begin[P.B] = slots;
   dp.batch = P.B;
   dp.n_heads = P.H;
   dp.total_tiles = T;

@@ -65,6 +65,11 @@ struct DecodeParams {
   // ones (sequence b's tiles are [tile128_begin[b], tile128_begin[b + 1]))
   int32_t tile128_begin[HS2_MAX_BATCH + 1];
   int32_t total_tiles128;
+  // pass 1 with CTAs of each sequence's own (seq_split): sequence b owns CTAs
+  // [cta_begin[b], cta_begin[b + 1]), which split its tiles equally, and the partial slot of a
+  // CTA is its index; otherwise CTA i owns tiles [i T / G, (i + 1) T / G) of all sequences
+  int32_t seq_split;
+  int32_t cta_begin[HS2_MAX_BATCH + 1];
 };
 
 // Chunk / prefill (n_q > 1). Pass 1: blocks of 128 (query, head) rows (128 / H queries);
