@@ -478,39 +478,69 @@ def measure_block(a, w, hs2, dev, local, pg, world):
     # ---- end to end through the public API: host queries in, host results out, every step
     e2e = None
     if not a.no_e2e:
-        # one pinned host buffer in and one out per step: the queries of every layer packed
-        # together, and the outputs, indices and counts written into one device buffer
+        # One pinned host buffer in and one out per step: the queries of every layer packed
+        # together, and the outputs, indices and counts written into one device buffer. Two
+        # device slots let the copies of one step overlap the kernels of another, as a serving
+        # loop would: step k's queries go into slot k % 2 on a copy stream while step k - 1
+        # computes, the block waits for them, and its results return on the copy stream once
+        # the block has ended. A slot is refilled only after the block that read it has ended,
+        # and only after its previous results have been copied out.
         qn = d["q_full"].numel()
         hq_all = torch.cat([d["q_full"].reshape(-1)] + [q.reshape(-1) for q in d["q_sparse"]]) \
             .cpu().pin_memory()
-        dq_all = torch.empty_like(hq_all, device=dev)
-        dq = dq_all[:qn].view(d["q_full"].shape)
-        dqs = [dq_all[(l + 1) * qn:(l + 2) * qn].view(d["q_sparse"][l].shape) for l in range(L)]
         on = out.numel()
         o_bytes, i_bytes, c_bytes = (1 + L) * on * 2, idx.numel() * 4, cnt.numel() * 4
-        dbuf = torch.empty(o_bytes + i_bytes + c_bytes, dtype=torch.uint8, device=dev)
-        o_all = dbuf[:o_bytes].view(torch.bfloat16)
-        eo = o_all[:on].view(out.shape)
-        eos = [o_all[(l + 1) * on:(l + 2) * on].view(out.shape) for l in range(L)]
-        eidx = dbuf[o_bytes:o_bytes + i_bytes].view(torch.int32).view(idx.shape)
-        ecnt = dbuf[o_bytes + i_bytes:].view(torch.int32).view(cnt.shape)
-        hbuf = torch.empty(dbuf.numel(), dtype=torch.uint8).pin_memory()
+        slots = []
+        for _ in range(2):
+            dq_all = torch.empty_like(hq_all, device=dev)
+            dbuf = torch.empty(o_bytes + i_bytes + c_bytes, dtype=torch.uint8, device=dev)
+            o_all = dbuf[:o_bytes].view(torch.bfloat16)
+            slots.append(dict(
+                dq_all=dq_all, dbuf=dbuf,
+                dq=dq_all[:qn].view(d["q_full"].shape),
+                dqs=[dq_all[(l + 1) * qn:(l + 2) * qn].view(d["q_sparse"][l].shape) for l in range(L)],
+                eo=o_all[:on].view(out.shape),
+                eos=[o_all[(l + 1) * on:(l + 2) * on].view(out.shape) for l in range(L)],
+                eidx=dbuf[o_bytes:o_bytes + i_bytes].view(torch.int32).view(idx.shape),
+                ecnt=dbuf[o_bytes + i_bytes:].view(torch.int32).view(cnt.shape),
+                hbuf=torch.empty(dbuf.numel(), dtype=torch.uint8).pin_memory()))
         h2d = hq_all.numel() * 2
-        d2h = hbuf.numel()
+        d2h = slots[0]["hbuf"].numel()
+        cstream = torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = torch.cuda.Event()
 
-        def e2e_step():
-            dq_all.copy_(hq_all, non_blocking=True)
-            hs2.block_decode(cache, dq, dqs, eo, eos, lse, scores, eidx, ecnt, ws,
-                             topk=w.topk, window=w.window)
-            hbuf.copy_(dbuf, non_blocking=True)
+        def e2e_run(n, start=None):
+            """n pipelined steps; returns after enqueueing them (stream waits for the last copy)."""
+            if start is not None:
+                cstream.wait_event(start)
+            with torch.cuda.stream(cstream):
+                slots[0]["dq_all"].copy_(hq_all, non_blocking=True)
+                ev_in[0].record(cstream)
+            for k in range(n):
+                sk, sl = k % 2, slots[k % 2]
+                stream.wait_event(ev_in[sk])
+                hs2.block_decode(cache, sl["dq"], sl["dqs"], sl["eo"], sl["eos"], lse, scores,
+                                 sl["eidx"], sl["ecnt"], ws, topk=w.topk, window=w.window)
+                ev_done[sk].record(stream)
+                with torch.cuda.stream(cstream):
+                    if k + 1 < n:   # the next step's queries, into the slot step k - 1 read
+                        if k >= 1:
+                            cstream.wait_event(ev_done[1 - sk])
+                        slots[1 - sk]["dq_all"].copy_(hq_all, non_blocking=True)
+                        ev_in[1 - sk].record(cstream)
+                    cstream.wait_event(ev_done[sk])
+                    sl["hbuf"].copy_(sl["dbuf"], non_blocking=True)
+            ev_out.record(cstream)
+            stream.wait_event(ev_out)
 
-        for _ in range(3):
-            e2e_step()
+        e2e_run(3)
+        torch.cuda.synchronize()
         barrier()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        for _ in range(a.steps):
-            e2e_step()
+        e2e_run(a.steps, start=a0)
         a1.record(stream)
         torch.cuda.synchronize()
         barrier()
