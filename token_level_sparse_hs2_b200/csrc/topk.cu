@@ -550,16 +550,35 @@ __global__ void __launch_bounds__(kThreadsTk, kRegs ? 1 : 2) topk_select_kernel(
         sm.seg_src[threadIdx.x] = info.x;
       }
       __syncthreads();
-      for (int j = threadIdx.x; j < n; j += kThreadsTk) {
-        int lo = 0, hi = ns - 1;   // the last segment starting at or before j
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (sm.seg_pre[mid] <= j) lo = mid;
-          else hi = mid - 1;
+      // every thread's loads in flight at once (up to kCandCap / kThreadsTk each), then stored
+      // (the many-rows variant, held to 64 registers, keeps one load pair at a time)
+      constexpr int kPer = kRegs ? kCandCap / kThreadsTk : 1;
+      uint32_t kk[kPer];
+      int32_t ii[kPer];
+      for (int j0 = 0; j0 < n; j0 += kPer * kThreadsTk) {
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+          const int j = j0 + q * kThreadsTk + threadIdx.x;
+          if (j < n) {
+            int lo = 0, hi = ns - 1;   // the last segment starting at or before j
+            while (lo < hi) {
+              const int mid = (lo + hi + 1) >> 1;
+              if (sm.seg_pre[mid] <= j) lo = mid;
+              else hi = mid - 1;
+            }
+            const int src = sm.seg_src[lo] + (j - sm.seg_pre[lo]);
+            kk[q] = __ldcg(gkey + src);
+            ii[q] = __ldcg(gidx + src);
+          }
         }
-        const int src = sm.seg_src[lo] + (j - sm.seg_pre[lo]);
-        sm.key[j] = __ldcg(gkey + src);
-        sm.idx[j] = __ldcg(gidx + src);
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+          const int j = j0 + q * kThreadsTk + threadIdx.x;
+          if (j < n) {
+            sm.key[j] = kk[q];
+            sm.idx[j] = ii[q];
+          }
+        }
       }
     }
     __syncthreads();
