@@ -7,8 +7,8 @@
 // s[t] = sum_h exp(c q_h . k_t - lse_h), lse_h from the output pass. With MQA ("HySparse2:
 // Hybrid Sparse Attention with Two-Level KV Sharing", "Inference cost") every 128-row K tile
 // meets all H query heads in one tensor-core product, D = K_tile . Q^T (M = 128 tokens,
-// N = H heads), so one thread of the epilogue owns one token and sums its H exponentials
-// without any exchange between threads.
+// N = H heads, or 2H query terms for e4m3 below), so one thread of the epilogue owns one
+// token and sums its H exponentials without any exchange between threads.
 //
 // Cache formats:
 //  * bf16: kind::f16 products over two 64-dim halves of the tile (8 steps of K = 16).
